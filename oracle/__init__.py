@@ -1,0 +1,130 @@
+"""fp64 CPU oracle for the gated delta rule.
+
+TEST INFRASTRUCTURE ONLY: tests/, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product path (``gated_delta_rule_59_b200``) never imports it, and
+nothing here imports the product path.
+
+Contents
+  run(...)         token-by-token fp64 recurrence (C library ``liboracle.so``),
+                   three independent update forms (see ``dr_oracle.c``).
+  chunk_ref        numpy fp64 chunk (UT/WY) form, used to pin the chunk algebra.
+  brute            exact rational brute force on tiny inputs.
+
+Parity pins live in ``tests/test_oracle_*.py``.  Every function here is pinned:
+the three forms against one another, against exact rational arithmetic
+(``brute``), against closed forms (scalar recurrence, orthonormal-key recall,
+Householder norm preservation) and invariants (beta = 0, g = 0, linearity).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dr_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` with gcc (OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+        os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)
+    ):
+        cmd = [
+            "gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+            "-std=c11", "-Wall", "-o", _LIB_PATH, _SRC, "-lm",
+        ]
+        subprocess.run(cmd, check=True)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int32)
+        lib.oracle_run.argtypes = [
+            dp, dp, dp, dp, dp, dp, ip,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int,
+            dp, dp,
+        ]
+        lib.oracle_run.restype = ctypes.c_int
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor on the CPU
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a, typ=ctypes.c_double):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(typ))
+
+
+def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
+        form: int = 2, threads: int = 0):
+    """Token-by-token fp64 recurrence.
+
+    q, k: [B, T, Hqk, dk]; v: [B, T, Hv, dv]; g, beta: [B, T, Hv] (g may be None);
+    state_in: [N, Hv, dk, dv] or None (zeros); cu_seqlens: int [N+1] or None.
+    Returns (o [B, T, Hv, dv], state_out [N, Hv, dk, dv]) as float64 numpy arrays.
+    """
+    lib = _load()
+    q, k, v, g, beta, state_in = (_f64(a) for a in (q, k, v, g, beta, state_in))
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    assert k.shape == q.shape and v.shape[:2] == (B, T) and beta.shape == (B, T, Hv)
+    if g is not None:
+        assert g.shape == (B, T, Hv)
+    cu = None
+    if cu_seqlens is not None:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        N = cu.shape[0] - 1
+    else:
+        N = B
+    if state_in is not None:
+        assert state_in.shape == (N, Hv, dk, dv), state_in.shape
+    o = np.zeros((B, T, Hv, dv), dtype=np.float64)
+    st = np.zeros((N, Hv, dk, dv), dtype=np.float64)
+    rc = lib.oracle_run(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
+        _ptr(cu, ctypes.c_int32), N, B, T, Hqk, Hv, dk, dv, float(scale), int(form),
+        int(threads), _ptr(o), _ptr(st),
+    )
+    if rc != 0:
+        raise ValueError(f"oracle_run failed with code {rc}")
+    return o, st
+
+
+def step(q, k, v, g, beta, state, scale: float = 1.0, form: int = 2, threads: int = 0):
+    """One decode step (T = 1) for every (batch, v-head).
+
+    q, k: [B, Hqk, dk]; v: [B, Hv, dv]; g, beta: [B, Hv]; state: [B, Hv, dk, dv].
+    Returns (o [B, Hv, dv], new_state [B, Hv, dk, dv]); ``state`` is not modified.
+    """
+    q, k, v, beta, state = (_f64(a) for a in (q, k, v, beta, state))
+    g = _f64(g)
+    o, st = run(q[:, None], k[:, None], v[:, None], None if g is None else g[:, None],
+                beta[:, None], state, None, scale, form, threads)
+    return o[:, 0], st
