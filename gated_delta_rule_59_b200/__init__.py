@@ -1,0 +1,177 @@
+"""B200 gated delta rule: thin Python binding over the C ABI of ``libdr.so``.
+
+This module only marshals arguments: it checks tensor placement, dtype and
+contiguity, allocates outputs with PyTorch (device memory and streams are the
+only things PyTorch does here) and passes raw device pointers plus the current
+CUDA stream to ``dr_chunk_fwd`` / ``dr_recurrent_step`` (``include/dr.h``).
+Every step of the recurrence runs in the library's CUDA kernels; there is no
+CPU or PyTorch fallback, and a missing or unloadable ``libdr.so`` raises.
+
+    o, state_out = chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None)
+    o = recurrent_step(q, k, v, g, beta, state)      # state updated in place
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = ["chunk_fwd", "recurrent_step", "device_status", "prefill_kernel", "lib", "DrError",
+           "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdr.so")
+
+DR_F32, DR_BF16 = 0, 1
+_DTYPES = {torch.float32: DR_F32, torch.bfloat16: DR_BF16}
+STATUS = {0: "DR_OK", 1: "DR_ERR_NULL", 2: "DR_ERR_SHAPE", 3: "DR_ERR_DTYPE", 4: "DR_ERR_ALIGN",
+          5: "DR_ERR_UNSUPPORTED", 6: "DR_ERR_CUDA", 7: "DR_ERR_TIMEOUT"}
+
+_lib = None
+
+
+class DrError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({_status_string(code)})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libdr.so`` (built in-tree by ``gated_delta_rule_59_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m gated_delta_rule_59_b200.build` "
+                "(there is no fallback implementation)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, fp, ip, i32 = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32
+        L.dr_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i32, i32, i32, i32, i32, i32,
+                                   ctypes.c_int, ctypes.c_float, vp, ctypes.c_int, fp, vp]
+        L.dr_chunk_fwd.restype = ctypes.c_int
+        L.dr_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, i32,
+                                        ctypes.c_int, ctypes.c_float, vp, ctypes.c_int, vp]
+        L.dr_recurrent_step.restype = ctypes.c_int
+        L.dr_status_string.argtypes = [ctypes.c_int]
+        L.dr_status_string.restype = ctypes.c_char_p
+        L.dr_get_device_status.argtypes = [vp]
+        L.dr_get_device_status.restype = ctypes.c_int
+        L.dr_version.restype = ctypes.c_int32
+        L.dr_chunk_fwd_kernel.argtypes = [ctypes.c_int, ctypes.c_int32, ctypes.c_int32]
+        L.dr_chunk_fwd_kernel.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _status_string(code: int) -> str:
+    try:
+        return lib().dr_status_string(code).decode()
+    except Exception:  # pragma: no cover - only while the library fails to load
+        return "?"
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtype=None, device=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
+              output_final_state: bool = True, out_dtype=torch.float32, o=None, state_out=None):
+    """Chunked prefill through ``dr_chunk_fwd``.
+
+    q, k [B, T, Hqk, dk] and v [B, T, Hv, dv] in bf16 or fp32 (same dtype);
+    g (or None), beta [B, T, Hv] fp32; state_in [N, Hv, dk, dv] fp32 or None;
+    cu_seqlens int32 [N+1] (device) or None.  Returns (o [B, T, Hv, dv] in
+    ``out_dtype``, state_out [N, Hv, dk, dv] fp32 or None).
+    """
+    if q.dtype not in _DTYPES or out_dtype not in _DTYPES:
+        raise ValueError("q/k/v must be bf16 or fp32; out_dtype bf16 or fp32")
+    dev = q.device
+    _check(q, "q", q.dtype, dev)
+    _check(k, "k", q.dtype, dev)
+    _check(v, "v", q.dtype, dev)
+    _check(g, "g", torch.float32, dev)
+    _check(beta, "beta", torch.float32, dev)
+    _check(state_in, "state_in", torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    if k.shape != q.shape or v.shape[:2] != (B, T) or beta.shape != (B, T, Hv):
+        raise ValueError("inconsistent shapes")
+    if g is not None and g.shape != (B, T, Hv):
+        raise ValueError("g must be [B, T, Hv]")
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if state_in is not None and tuple(state_in.shape) != (N, Hv, dk, dv):
+        raise ValueError(f"state_in must be {(N, Hv, dk, dv)}")
+    if o is None:
+        o = torch.empty((B, T, Hv, dv), dtype=out_dtype, device=dev)
+    _check(o, "o", out_dtype, dev)
+    if output_final_state and state_out is None:
+        state_out = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=dev)
+    _check(state_out, "state_out", torch.float32, dev)
+    rc = lib().dr_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), N,
+        B, T, Hqk, Hv, dk, dv, _DTYPES[q.dtype], float(scale), _ptr(o), _DTYPES[out_dtype],
+        _ptr(state_out), _stream(dev))
+    if rc != 0:
+        raise DrError(rc, "dr_chunk_fwd")
+    return o, state_out
+
+
+def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.float32, o=None):
+    """One decode step through ``dr_recurrent_step``; ``state`` is updated in place.
+
+    q, k [B, Hqk, dk], v [B, Hv, dv] (bf16 or fp32); g (or None), beta [B, Hv] fp32;
+    state [B, Hv, dk, dv] fp32.  Returns o [B, Hv, dv] in ``out_dtype``.
+    """
+    if q.dtype not in _DTYPES or out_dtype not in _DTYPES:
+        raise ValueError("q/k/v must be bf16 or fp32; out_dtype bf16 or fp32")
+    dev = q.device
+    for t, name, dt in ((q, "q", q.dtype), (k, "k", q.dtype), (v, "v", q.dtype),
+                        (g, "g", torch.float32), (beta, "beta", torch.float32),
+                        (state, "state", torch.float32)):
+        _check(t, name, dt, dev)
+    B, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    if tuple(state.shape) != (B, Hv, dk, dv) or beta.shape != (B, Hv):
+        raise ValueError("inconsistent shapes")
+    if o is None:
+        o = torch.empty((B, Hv, dv), dtype=out_dtype, device=dev)
+    _check(o, "o", out_dtype, dev)
+    rc = lib().dr_recurrent_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), B, Hqk, Hv, dk, dv,
+        _DTYPES[q.dtype], float(scale), _ptr(o), _DTYPES[out_dtype], _stream(dev))
+    if rc != 0:
+        raise DrError(rc, "dr_recurrent_step")
+    return o
+
+
+KERNELS = {0: None, 1: "simt_f32", 2: "tc_bf16"}
+
+
+def prefill_kernel(dtype, dk: int, dv: int):
+    """Name of the kernel dr_chunk_fwd picks for these inputs ('tc_bf16', 'simt_f32' or None)."""
+    return KERNELS[lib().dr_chunk_fwd_kernel(_DTYPES[dtype], dk, dv)]
+
+
+def device_status(device=None) -> int:
+    """Synchronise and return (and clear) the library's device status code."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return int(lib().dr_get_device_status(_stream(dev)))

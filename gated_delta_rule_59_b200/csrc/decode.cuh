@@ -1,0 +1,122 @@
+// decode.cuh -- fused decode step (one token per sequence), state updated in place.
+//
+// Operation ("linear_attention" page: token-by-token rule on a decode step,
+// cached state overwritten in place; "DeltaNet" page, "The Delta Rule":
+// retrieve-and-replace form):
+//     H' = alpha H;  v_old = H'^T k;  delta = beta (v - v_old)
+//     H  = H' + k delta^T;            o = H^T q = alpha H^T q + (q.k) delta
+// with H = S^T stored [dk, dv] fp32 (dv contiguous) per (batch, v-head).
+//
+// The step is bound by HBM: each (b, h) state is read once and written once
+// (2 * dk * dv * 4 bytes) against ~4 dk dv flops.  One CTA owns one (b, h)
+// state.  A warp covers one full 512-byte state row with 16-byte vector
+// accesses (perfectly coalesced), the CTA's 8 warps cover 8 rows per pass, and
+// each thread keeps its 16 x 4 state values in registers between the read and
+// the write: the state touches HBM exactly twice and never goes through shared
+// memory.  The two column reductions over dk (H^T k and H^T q) are per-thread
+// partial sums followed by one cross-warp pass through shared memory.
+#pragma once
+
+#include "dr_common.cuh"
+
+namespace dr {
+
+template <int DK, int DV>
+struct DecodeShape {
+  static constexpr int C4 = DV / 4;                            // float4 per state row
+  static constexpr int RP = (256 / C4 < DK) ? 256 / C4 : DK;   // rows covered per pass
+  static constexpr int NT = C4 * RP;                           // threads per CTA
+  static constexpr int RPT = DK / RP;                          // rows per thread
+  static_assert(DV % 4 == 0 && DK % RP == 0, "unsupported decode shape");
+};
+
+template <int DK, int DV, typename Tin, typename Tout>
+__global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
+    decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
+                       const Tin *__restrict__ v, const float *__restrict__ g,
+                       const float *__restrict__ beta, float *__restrict__ state, int Hqk,
+                       int Hv, float scale, Tout *__restrict__ o) {
+  using S = DecodeShape<DK, DV>;
+  constexpr int C4 = S::C4, RP = S::RP, NT = S::NT, RPT = S::RPT;
+  __shared__ float ks[DK], qs[DK];
+  __shared__ float4 red_k[RP][C4], red_q[RP][C4];
+  __shared__ float qk_shared;
+
+  const int unit = blockIdx.x;  // b * Hv + h
+  const int b = unit / Hv, h = unit - (unit / Hv) * Hv;
+  const int hq = h / (Hv / Hqk);
+  const int t = threadIdx.x, c4 = t % C4, r0 = t / C4;
+
+  float4 *H = reinterpret_cast<float4 *>(state + (size_t)unit * DK * DV);
+  // Issue every state load first: RPT independent 16-byte loads per thread.
+  float4 hr[RPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) hr[i] = __ldcs(&H[(size_t)(r0 + i * RP) * C4 + c4]);
+
+  const size_t qk_off = ((size_t)b * Hqk + hq) * DK;
+  for (int i = t; i < DK; i += NT) {
+    ks[i] = io<Tin>::ld(k + qk_off + i);
+    qs[i] = scale * io<Tin>::ld(q + qk_off + i);
+  }
+  __syncthreads();
+  if (t < 32) {
+    float acc = 0.f;
+    for (int i = t; i < DK; i += 32) acc += ks[i] * qs[i];
+    acc = warp_sum(acc);
+    if (t == 0) qk_shared = acc;
+  }
+  float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const float kr = ks[r0 + i * RP], qr = qs[r0 + i * RP];
+    pk.x += kr * hr[i].x; pk.y += kr * hr[i].y; pk.z += kr * hr[i].z; pk.w += kr * hr[i].w;
+    pq.x += qr * hr[i].x; pq.y += qr * hr[i].y; pq.z += qr * hr[i].z; pq.w += qr * hr[i].w;
+  }
+  red_k[r0][c4] = pk;
+  red_q[r0][c4] = pq;
+  __syncthreads();
+  float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sq = sk;
+#pragma unroll 8
+  for (int r = 0; r < RP; ++r) {
+    const float4 a = red_k[r][c4], c = red_q[r][c4];
+    sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
+    sq.x += c.x; sq.y += c.y; sq.z += c.z; sq.w += c.w;
+  }
+  const float alpha = g ? expf(g[unit]) : 1.f;
+  const float bt = beta[unit];
+  const size_t vo = (size_t)unit * DV + 4 * c4;
+  float4 d;
+  d.x = bt * (io<Tin>::ld(v + vo + 0) - alpha * sk.x);
+  d.y = bt * (io<Tin>::ld(v + vo + 1) - alpha * sk.y);
+  d.z = bt * (io<Tin>::ld(v + vo + 2) - alpha * sk.z);
+  d.w = bt * (io<Tin>::ld(v + vo + 3) - alpha * sk.w);
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    const float kr = ks[r0 + i * RP];
+    float4 nh;
+    nh.x = alpha * hr[i].x + kr * d.x;
+    nh.y = alpha * hr[i].y + kr * d.y;
+    nh.z = alpha * hr[i].z + kr * d.z;
+    nh.w = alpha * hr[i].w + kr * d.w;
+    __stcs(&H[(size_t)(r0 + i * RP) * C4 + c4], nh);
+  }
+  if (r0 == 0) {
+    const float qk = qk_shared;
+    io<Tout>::st(o + vo + 0, alpha * sq.x + qk * d.x);
+    io<Tout>::st(o + vo + 1, alpha * sq.y + qk * d.y);
+    io<Tout>::st(o + vo + 2, alpha * sq.z + qk * d.z);
+    io<Tout>::st(o + vo + 3, alpha * sq.w + qk * d.w);
+  }
+}
+
+template <int DK, int DV, typename Tin, typename Tout>
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, float *state, int B, int Hqk, int Hv, float scale,
+                          void *o, cudaStream_t stream) {
+  const unsigned units = (unsigned)B * (unsigned)Hv;
+  decode_step_kernel<DK, DV, Tin, Tout><<<units, DecodeShape<DK, DV>::NT, 0, stream>>>(
+      (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, Hqk, Hv, scale, (Tout *)o);
+  return cudaGetLastError();
+}
+
+}  // namespace dr

@@ -1,0 +1,161 @@
+// dr_lib.cu -- the C ABI of libdr.so (declared in include/dr.h).
+//
+// Host side only: argument validation (before anything is launched), dtype and
+// head-dimension dispatch, launch on the caller's stream, status mapping.  All
+// kernels are compiled into this one translation unit so that they share the
+// device status word without relocatable device code.
+#include <cmath>
+#include <cstdint>
+
+#include "dr.h"
+#include "dr_common.cuh"
+#include "decode.cuh"
+#include "chunk_simt.cuh"
+#include "chunk_tc.cuh"
+
+#define DR_VERSION_NUMBER 100  // 0.1.0
+
+namespace {
+
+bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool dtype_ok(dr_dtype t) { return t == DR_F32 || t == DR_BF16; }
+
+template <typename Tin, typename Tout>
+cudaError_t decode_dispatch(int dk, int dv, const void *q, const void *k, const void *v,
+                            const float *g, const float *beta, float *state, int B, int Hqk,
+                            int Hv, float scale, void *o, cudaStream_t s) {
+#define DR_DEC(DK, DV)                                                                  \
+  if (dk == DK && dv == DV)                                                             \
+    return dr::launch_decode<DK, DV, Tin, Tout>(q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s);
+#define DR_DEC_ROW(DK) DR_DEC(DK, 16) DR_DEC(DK, 32) DR_DEC(DK, 64) DR_DEC(DK, 128)
+  DR_DEC_ROW(16) DR_DEC_ROW(32) DR_DEC_ROW(64) DR_DEC_ROW(128)
+#undef DR_DEC_ROW
+#undef DR_DEC
+  return cudaErrorInvalidValue;
+}
+
+template <typename Tin, typename Tout>
+cudaError_t simt_dispatch(int dk, int dv, const dr::PrefillArgs &a, int N, cudaStream_t s) {
+#define DR_SIMT(DK, DV) \
+  if (dk == DK && dv == DV) return dr::launch_chunk_simt<DK, DV, Tin, Tout>(a, N, s);
+#define DR_SIMT_ROW(DK) DR_SIMT(DK, 16) DR_SIMT(DK, 32) DR_SIMT(DK, 64) DR_SIMT(DK, 128)
+  DR_SIMT_ROW(16) DR_SIMT_ROW(32) DR_SIMT_ROW(64) DR_SIMT_ROW(128)
+#undef DR_SIMT_ROW
+#undef DR_SIMT
+  return cudaErrorInvalidValue;
+}
+
+template <typename Tin>
+cudaError_t simt_dispatch_out(dr_dtype od, int dk, int dv, const dr::PrefillArgs &a, int N,
+                              cudaStream_t s) {
+  return od == DR_F32 ? simt_dispatch<Tin, float>(dk, dv, a, N, s)
+                      : simt_dispatch<Tin, __nv_bfloat16>(dk, dv, a, N, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *state_in, const int32_t *cu_seqlens,
+                       int32_t n_seqs, int32_t B, int32_t T, int32_t Hqk, int32_t Hv,
+                       int32_t dk, int32_t dv, dr_dtype in_dtype, float scale, void *o,
+                       dr_dtype o_dtype, float *state_out, dr_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return DR_ERR_DTYPE;
+  if (B < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return DR_ERR_SHAPE;
+  if (Hv % Hqk != 0) return DR_ERR_SHAPE;
+  if (cu_seqlens && (B != 1 || n_seqs < 0)) return DR_ERR_SHAPE;
+  if (!dim_ok(dk) || !dim_ok(dv)) return DR_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return DR_ERR_UNSUPPORTED;
+  const int64_t N = cu_seqlens ? n_seqs : B;
+  const bool tokens = (int64_t)B * T > 0;
+  if (tokens && (!q || !k || !v || !beta || !o)) return DR_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(g, 4) ||
+      !aligned(beta, 4) || !aligned(cu_seqlens, 4))
+    return DR_ERR_ALIGN;
+  if (N == 0) return DR_OK;
+  if (N * Hv > 0x7fffffff) return DR_ERR_UNSUPPORTED;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  dr::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, (int)N, B, T, Hqk, Hv,
+                    scale, o, state_out};
+  cudaError_t e;
+  if (in_dtype == DR_BF16 && dr::tc_supported(dk, dv)) {
+    e = dr::tc_dispatch(dk, dv, o_dtype == DR_F32, a, (int)N, s);
+  } else if (in_dtype == DR_F32) {
+    e = simt_dispatch_out<float>(o_dtype, dk, dv, a, (int)N, s);
+  } else {
+    e = simt_dispatch_out<__nv_bfloat16>(o_dtype, dk, dv, a, (int)N, s);
+  }
+  return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
+dr_status dr_recurrent_step(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float *state, int32_t B, int32_t Hqk,
+                            int32_t Hv, int32_t dk, int32_t dv, dr_dtype in_dtype,
+                            float scale, void *o, dr_dtype o_dtype, dr_stream stream) {
+  if (!dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return DR_ERR_DTYPE;
+  if (B < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return DR_ERR_SHAPE;
+  if (Hv % Hqk != 0) return DR_ERR_SHAPE;
+  if (!dim_ok(dk) || !dim_ok(dv)) return DR_ERR_UNSUPPORTED;
+  if (!std::isfinite(scale)) return DR_ERR_UNSUPPORTED;
+  if (B == 0) return DR_OK;
+  if (!q || !k || !v || !beta || !state || !o) return DR_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(state, 16) || !aligned(g, 4) || !aligned(beta, 4))
+    return DR_ERR_ALIGN;
+  if ((int64_t)B * Hv > 0x7fffffff) return DR_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (in_dtype == DR_BF16)
+    e = o_dtype == DR_F32
+            ? decode_dispatch<__nv_bfloat16, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s)
+            : decode_dispatch<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s);
+  else
+    e = o_dtype == DR_F32
+            ? decode_dispatch<float, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s)
+            : decode_dispatch<float, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s);
+  return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
+dr_kernel dr_chunk_fwd_kernel(dr_dtype in_dtype, int32_t dk, int32_t dv) {
+  if (!dtype_ok(in_dtype) || !dim_ok(dk) || !dim_ok(dv)) return DR_KERNEL_NONE;
+  if (in_dtype == DR_BF16 && dr::tc_supported(dk, dv)) return DR_KERNEL_TC_BF16;
+  return DR_KERNEL_SIMT_F32;
+}
+
+const char *dr_status_string(dr_status status) {
+  switch (status) {
+    case DR_OK: return "ok";
+    case DR_ERR_NULL: return "a required pointer is NULL";
+    case DR_ERR_SHAPE: return "inconsistent or invalid sizes";
+    case DR_ERR_DTYPE: return "unknown dtype";
+    case DR_ERR_ALIGN: return "pointer not aligned (16 bytes for tensors, 4 for g/beta/cu_seqlens)";
+    case DR_ERR_UNSUPPORTED: return "unsupported head dimension or argument";
+    case DR_ERR_CUDA: return "CUDA runtime error";
+    case DR_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+  }
+  return "unknown status";
+}
+
+dr_status dr_get_device_status(dr_stream stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DR_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpyFromSymbol(&word, dr::g_device_status, sizeof(int)) != cudaSuccess)
+    return DR_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(dr::g_device_status, &zero, sizeof(int)) != cudaSuccess)
+      return DR_ERR_CUDA;
+  }
+  if (word & (1 << DR_ERR_TIMEOUT)) return DR_ERR_TIMEOUT;
+  if (word & (1 << DR_ERR_SHAPE)) return DR_ERR_SHAPE;
+  return DR_OK;
+}
+
+int32_t dr_version(void) { return DR_VERSION_NUMBER; }
+
+}  // extern "C"

@@ -1,0 +1,140 @@
+/*
+ * dr.h -- C ABI of the B200 gated delta-rule library (libdr.so).
+ *
+ * The operation (per sequence n and value head h, query/key head
+ * hq = h / (Hv / Hqk)):
+ *
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t (scale * q_t),          alpha_t = exp(g_t)
+ *
+ * - update of the "DeltaNet Attention" page (class docstring); its error-correction
+ *   and retrieve-and-replace forms are on the "DeltaNet" page ("The Delta Rule");
+ * - gate (decays), write strength (betas), head layout and state_input semantics
+ *   of the "linear_attention" page (LinearAttention): decays are float32 log
+ *   kept-fractions, betas are in (0, 1) or (0, 2), the query reads the updated
+ *   state, and the state is one key_dim x value_dim matrix per head.
+ *
+ * State is stored as H = S^T:  [.., dk, dv] float32, row-major (dv contiguous).
+ *
+ * Conventions for every call
+ * - All tensor pointers are DEVICE memory owned by the caller.  The library
+ *   never allocates device memory and never frees.  Tensors are dense, row-major
+ *   and contiguous in the layouts below.
+ * - q, k, v, o, state_in, state_out and state must be 16-byte aligned; g and beta
+ *   4-byte aligned; cu_seqlens 4-byte aligned.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *   Argument errors are detected on the host before anything is launched and
+ *   leave every output untouched.  A failed launch returns DR_ERR_CUDA.
+ * - Errors the host cannot see (malformed cu_seqlens contents, a bounded
+ *   device-side wait that ran out) set a device status word instead: the kernel
+ *   skips the affected work unit, and dr_get_device_status() reports it.
+ * - Supported: dk, dv in {16, 32, 64, 128}; Hv % Hqk == 0 (GQA: value head h uses
+ *   query/key head h / (Hv / Hqk)); scale is any finite float (1.0 = o = S q).
+ * - No call throws, exits or keeps mutable host state; calls are thread-safe.
+ */
+#ifndef DR_H
+#define DR_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DR_API __attribute__((visibility("default")))
+#else
+#define DR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DR_OK = 0,
+  DR_ERR_NULL = 1,        /* a required pointer is NULL                          */
+  DR_ERR_SHAPE = 2,       /* inconsistent or negative sizes (incl. Hv % Hqk != 0) */
+  DR_ERR_DTYPE = 3,       /* unknown dtype code                                  */
+  DR_ERR_ALIGN = 4,       /* a pointer violates the alignment rule above          */
+  DR_ERR_UNSUPPORTED = 5, /* valid but unsupported (e.g. dk = 96)                 */
+  DR_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed                 */
+  DR_ERR_TIMEOUT = 7      /* a bounded device-side wait gave up                   */
+} dr_status;
+
+typedef enum { DR_F32 = 0, DR_BF16 = 1 } dr_dtype;
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *dr_stream;
+
+/*
+ * dr_chunk_fwd -- prompt (prefill) pass: the "chunked rule on a prompt" of the
+ * "linear_attention" page, computed chunkwise in the UT/WY form of
+ * "Parallelizing Linear Transformers with the Delta Rule over Sequence Length"
+ * (the reference both DeltaNet pages cite), 64-token chunks, decays folded in.
+ *
+ *   q, k       [B, T, Hqk, dk]   in_dtype (DR_BF16 or DR_F32), L2-normalised by the caller
+ *   v          [B, T, Hv, dv]    in_dtype
+ *   g          [B, T, Hv] f32    log decay (<= 0 expected); NULL => no decay (plain DeltaNet)
+ *   beta       [B, T, Hv] f32    write strength
+ *   state_in   [N, Hv, dk, dv] f32 or NULL (=> zero state: a fresh prompt).  Read only.
+ *   cu_seqlens device int32 [n_seqs + 1] or NULL.  If given, B must be 1, N = n_seqs,
+ *              sequence n is tokens [cu_seqlens[n], cu_seqlens[n+1]) with
+ *              cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_seqs] = T (checked on
+ *              the device: a violation skips that sequence and sets DR_ERR_SHAPE
+ *              in the device status).  If NULL, N = B sequences of T tokens.
+ *   o          [B, T, Hv, dv]    o_dtype (DR_F32 or DR_BF16); every token's output is written
+ *   state_out  [N, Hv, dk, dv] f32 or NULL (=> final state not returned).  It may be
+ *              state_in itself (in-place update); a partial overlap is undefined.
+ *   T = 0 or N = 0 is valid: nothing is read from q/k/v; state_out (if given) receives
+ *   state_in (or zeros).
+ */
+DR_API dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *state_in,
+                              const int32_t *cu_seqlens, int32_t n_seqs, int32_t B, int32_t T,
+                              int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv,
+                              dr_dtype in_dtype, float scale, void *o, dr_dtype o_dtype,
+                              float *state_out, dr_stream stream);
+
+/* Which prefill kernel dr_chunk_fwd launches for these inputs (host only, no device call). */
+typedef enum {
+  DR_KERNEL_NONE = 0,     /* unsupported dtype / head dimensions                  */
+  DR_KERNEL_SIMT_F32 = 1, /* CUDA-core kernel, fp32 arithmetic                    */
+  DR_KERNEL_TC_BF16 = 2   /* tcgen05 tensor-core kernel, bf16 operands, fp32 state */
+} dr_kernel;
+DR_API dr_kernel dr_chunk_fwd_kernel(dr_dtype in_dtype, int32_t dk, int32_t dv);
+
+/*
+ * dr_recurrent_step -- one decode token per sequence: the "token-by-token rule on
+ * a decode step" of the "linear_attention" page, with the cache overwritten in
+ * place (state_input semantics there).  Computed as
+ *     H' = alpha H;  v_old = H'^T k;  delta = beta (v - v_old);
+ *     H  = H' + k delta^T (in place);  o = H^T (scale q)
+ * which is the retrieve-and-replace form of the "DeltaNet" page ("The Delta Rule").
+ *
+ *   q, k   [B, Hqk, dk] in_dtype;   v [B, Hv, dv] in_dtype
+ *   g      [B, Hv] f32 or NULL;     beta [B, Hv] f32
+ *   state  [B, Hv, dk, dv] f32, read and overwritten in place
+ *   o      [B, Hv, dv] o_dtype
+ */
+DR_API dr_status dr_recurrent_step(const void *q, const void *k, const void *v,
+                                   const float *g, const float *beta, float *state, int32_t B,
+                                   int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv,
+                                   dr_dtype in_dtype, float scale, void *o, dr_dtype o_dtype,
+                                   dr_stream stream);
+
+/* Static English description of a status code (never NULL). */
+DR_API const char *dr_status_string(dr_status status);
+
+/*
+ * Synchronises `stream`, then reports and clears the device status word of the
+ * current device: DR_OK, DR_ERR_SHAPE (bad cu_seqlens contents) or
+ * DR_ERR_TIMEOUT (a bounded device wait gave up).  DR_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+DR_API dr_status dr_get_device_status(dr_stream stream);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+DR_API int32_t dr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DR_H */
