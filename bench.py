@@ -312,7 +312,7 @@ def run_ours(args, dist: Dist):
     }
     line.update(secondary)
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(host, n_tok=2048)
+        line["cpu_baseline"] = cpu_baseline(host, n_tok=host.q.shape[1])
     del p, o, st, flush
     dist.close()
     if dist.rank == 0:
