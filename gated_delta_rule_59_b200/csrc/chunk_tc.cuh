@@ -10,32 +10,35 @@
 //   O = diag(gamma) Q H0 + (Gamma * Q K^T * incl_lower) Delta
 //   H = gamma_C H0 + Ktil^T Delta,  Ktil_s = e^{b_C - b_s} k_s
 //
-// B200 mapping (one CTA of 256 threads per (sequence, v-head); the recurrence
-// over chunks is sequential inside the CTA):
-//  * Every matrix product is a tcgen05.mma (bf16 operands from shared memory,
-//    fp32 accumulators in TMEM), issued by one thread.  All products are
-//    arranged with M = 128 so the tensor core runs its full-width shape:
-//        G     = [K; Q] K^T                 (rows 0-63: K K^T, 64-127: Q K^T)
-//        W^T   = K^T (T diag(beta gamma))^T,  U^T = V^T (T diag(beta))^T
-//        Delta^T = U^T + H0^T (-W^T)        (accumulates onto U^T in TMEM)
-//        Oa    = H0^T Q^T,   Ob = Delta^T P^T   (O^T = diag(gamma) Oa + Ob)
-//        Hupd  = Delta~^T K   with Delta~_s = e^{b_C - b_s} Delta_s
-//  * The fp32 master state lives in registers (thread = one TMEM lane = one
-//    value column j, 64 of the dk rows per warpgroup); a bf16 copy of H0^T in
-//    shared memory is the MMA operand.  Each chunk the state update
-//    H = gamma_C H + Hupd is done in registers from the TMEM accumulator.
-//  * Q, K, V chunks arrive by TMA (128-byte swizzle, no multicast) one chunk
-//    ahead into a second buffer.  Sequence starts need no alignment: rows past
-//    the end of a sequence are neutralised by beta = g = 0.
-//  * T = (I + L)^-1 is inverted in fp32 in shared memory by blocked forward
-//    substitution (16x16 diagonal blocks, then three block-merge rounds).
-//  * Precision: operands computed in fp32 inside the kernel (T diag(beta),
-//    T diag(beta gamma), P, Delta, Delta~) are fed to the tensor core as a
-//    bf16 pair x = hi + lo (hi = bf16(x), lo = bf16(x - hi)), two MMAs into the
-//    same accumulator (three for P Delta, dropping lo x lo).  A single bf16
-//    rounding of these (2^-8 relative) alone exceeds the 2e-2 max/RMS error
-//    budget on short sequences; the pair keeps ~2^-16.  Inputs (q, k, v) are
-//    exact in bf16; the H0 operand stays a single bf16 copy.
+// B200 mapping.  One CTA of 512 threads per (sequence, v-head); the chunk chain
+// is sequential inside the CTA, and the CTA is warp-specialised so that the
+// state-independent work of chunk c+1 runs under the state-dependent chain of
+// chunk c:
+//   warpgroup 0  warp 0: TMA producer (Q, K double-buffered; V single)
+//                warp 1: tcgen05.mma issuer (one thread)
+//                warp 2: gates: prefix sums of g, e^b, e^{b_C - b} per chunk
+//   warpgroup 1  "prep" (chunk c+1): L and P from the Gram MMA, the fp32
+//                triangular inverse T, the T diag(beta[gamma]) operands, -W^T
+//   warpgroups 2-3 "state" (chunk c): Delta epilogue, outputs, state update;
+//                the fp32 master state lives in their registers (thread = one
+//                TMEM lane = one value column j; 64 of the key rows each)
+// Every product is a tcgen05.mma with M = 128 (bf16 operands, fp32 TMEM
+// accumulators):
+//        G       = [K; Q] K^T                (rows 0-63: K K^T, 64-127: Q K^T)
+//        W^T     = K^T (T diag(beta gamma))^T,   U^T = V^T (T diag(beta))^T
+//        Delta^T = U^T + H0^T (-W^T)         (accumulates onto U^T in TMEM)
+//        Oa      = H0^T Q^T,   Ob = Delta^T P^T     (O^T = diag(gamma) Oa + Ob)
+//        Hupd    = Delta~^T K  with Delta~_s = e^{b_C - b_s} Delta_s
+// H0^T (bf16) is the A operand of two of them and is read from TMEM, written
+// there by the state warps each chunk.
+// Precision: operands computed in fp32 inside the kernel (T diag(beta),
+// T diag(beta gamma), P, Delta, Delta~) go to the tensor core as a bf16 pair
+// x = hi + lo (hi = bf16(x), lo = bf16(x - hi)): two MMAs into one accumulator
+// (three for P Delta, dropping lo x lo).  A single bf16 rounding of these
+// (2^-8 relative) alone exceeds the 2e-2 max/RMS error budget on short
+// sequences; the pair keeps ~2^-16.  q, k, v are exact in bf16.
+// Decays are always formed from differences of cumulative log decays, never as
+// ratios of separate exponentials (no overflow for strongly negative g).
 #pragma once
 
 #include <cuda.h>
@@ -48,51 +51,68 @@
 namespace dr {
 namespace tck {
 
-constexpr int C = 64, DK = 128, DV = 128, NT = 256;
+constexpr int C = 64, DK = 128, DV = 128, NT = 512;
 constexpr float LOG2E = 1.4426950408889634f;
 
-// shared-memory map (bytes from a 1024-aligned base).  Regions R1-R3 are reused
-// by operands whose lifetimes within a chunk do not overlap.
-constexpr uint32_t STAGE_BYTES = 49152;  // K0 Q0 K1 Q1 V0 V1, 8 KB each
-constexpr uint32_t OFF_K0 = 0, OFF_Q0 = 8192, OFF_K1 = 16384, OFF_Q1 = 24576;
-constexpr uint32_t OFF_V0 = 32768, OFF_V1 = 40960;
-constexpr uint32_t OFF_H = 2 * STAGE_BYTES;  // H0^T bf16, 2 x 16 KB (K-major, k = dk)
-constexpr uint32_t OFF_R1 = OFF_H + 32768;   // L fp32 [64][65]          | Delta^T lo
-constexpr uint32_t OFF_R2 = OFF_R1 + 17408;  // T fp32 [64][64] | -W^T   | Delta~^T lo
-constexpr uint32_t OFF_R3 = OFF_R2 + 16384;  // merge scratch | T diag(beta), T diag(beta gamma)
-                                             //   (hi, lo: 4 x 8 KB) | Delta^T hi, Delta~^T hi
-constexpr uint32_t OFF_R4 = OFF_R3 + 32768;  // P hi, P lo (8 KB each)
-constexpr uint32_t OFF_TB_H = OFF_R3, OFF_TB_L = OFF_R3 + 8192;
-constexpr uint32_t OFF_TBG_H = OFF_R3 + 16384, OFF_TBG_L = OFF_R3 + 24576;
-constexpr uint32_t OFF_W = OFF_R2;
-constexpr uint32_t OFF_D_H = OFF_R3, OFF_DT_H = OFF_R3 + 16384;
-constexpr uint32_t OFF_D_L = OFF_R1, OFF_DT_L = OFF_R2;
-constexpr uint32_t OFF_P_H = OFF_R4, OFF_P_L = OFF_R4 + 8192;
-constexpr uint32_t OFF_L = OFF_R1, OFF_T = OFF_R2, OFF_X = OFF_R3;
-constexpr uint32_t OFF_SMALL = OFF_R4 + 16384;
-constexpr uint32_t SMALL_BYTES = 4 * 64 * 4 + 64;
-constexpr uint32_t SMEM_BYTES = OFF_SMALL + SMALL_BYTES + 1024;  // + alignment slack
+// ---- shared memory (bytes from a 1024-aligned base) ----
+constexpr uint32_t QK_BYTES = 32768;                        // K0 Q0 K1 Q1, 8 KB boxes
+constexpr uint32_t QK_K0 = 0, QK_Q0 = 8192, QK_K1 = 16384, QK_Q1 = 24576;
+constexpr uint32_t OFF_QK = 0;                              // 2 stages
+constexpr uint32_t OFF_V = 2 * QK_BYTES;                    // V0, V1 (single stage)
+constexpr uint32_t V_BYTES = 16384;
+constexpr uint32_t OFF_RL = OFF_V + V_BYTES;                // L fp32 [64][65] | T diag(beta) hi, lo
+constexpr uint32_t OFF_RT = OFF_RL + 17408;                 // T fp32 [64][64] | -W^T bf16
+constexpr uint32_t OFF_RX = OFF_RT + 16384;                 // merge scratch | T diag(beta gamma) hi, lo
+constexpr uint32_t OFF_P = OFF_RX + 16384;                  // P hi, P lo
+constexpr uint32_t OFF_DH = OFF_P + 16384;                  // Delta^T hi
+constexpr uint32_t OFF_DL = OFF_DH + 16384;                 // Delta^T lo
+constexpr uint32_t OFF_DTH = OFF_DL + 16384;                // Delta~^T hi
+constexpr uint32_t OFF_DTL = OFF_DTH + 16384;               // Delta~^T lo
+constexpr uint32_t OFF_GATES = OFF_DTL + 16384;             // 2 slots x {bs2, beta, gam, dtil}[64]
+constexpr uint32_t OFF_BARS = OFF_GATES + 2 * 4 * 64 * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BARS + 256 + 1024;      // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_R2 % 1024 == 0 && OFF_R3 % 1024 == 0 && OFF_R4 % 1024 == 0, "tile alignment");
+static_assert(OFF_RL % 1024 == 0 && OFF_RT % 1024 == 0 && OFF_RX % 1024 == 0 &&
+                  OFF_P % 1024 == 0 && OFF_DH % 1024 == 0 && OFF_DTL % 1024 == 0,
+              "operand tiles must be 1024-byte aligned");
 
-// TMEM columns (fp32 accumulators, 128 lanes each)
-constexpr uint32_t COL_G = 0, COL_W = 64, COL_DU = 128, COL_OA = 192, COL_OB = 256, COL_HU = 320;
-constexpr uint32_t TMEM_COLS = 512;
+// ---- TMEM columns ----
+constexpr uint32_t COL_G = 0, COL_W = 64, COL_DU = 128, COL_OA = 192, COL_OB = 256;
+constexpr uint32_t COL_HU = 320, COL_H0 = 448, TMEM_COLS = 512;
 
-constexpr uint32_t ID_G = tc::idesc_bf16(128, 64, 0, 0);    // [K;Q] K^T
-constexpr uint32_t ID_MNK = tc::idesc_bf16(128, 64, 1, 0);  // K^T / V^T (MN-major A) x K-major B
-constexpr uint32_t ID_KMN64 = tc::idesc_bf16(128, 64, 0, 1);    // H0^T x (-W^T), MN-major B
+constexpr uint32_t ID_G = tc::idesc_bf16(128, 64, 0, 0);        // [K;Q] K^T
+constexpr uint32_t ID_MNK = tc::idesc_bf16(128, 64, 1, 0);      // K^T / V^T x T^T
+constexpr uint32_t ID_KMN64 = tc::idesc_bf16(128, 64, 0, 1);    // H0^T x (-W^T)
 constexpr uint32_t ID_KK64 = tc::idesc_bf16(128, 64, 0, 0);     // H0^T Q^T, Delta^T P^T
 constexpr uint32_t ID_KMN128 = tc::idesc_bf16(128, 128, 0, 1);  // Delta~^T K
 
-// Write 8 fp32 values as one 16-byte bf16 chunk of a swizzled 128-byte row.
+// ---- mbarriers ----
+enum Bar {
+  B_QK_FULL = 0,   // [2] TMA -> MMA
+  B_QK_EMPTY = 2,  // [2] MMA (after Hupd) -> TMA
+  B_V_FULL = 4,
+  B_V_EMPTY = 5,
+  B_GATE_FULL = 6,   // [2] gates warp (32) -> prep, state
+  B_GATE_EMPTY = 8,  // [2] prep (128) + state (256) -> gates warp
+  B_G_FULL = 10,     // MMA -> prep
+  B_G_EMPTY = 11,    // prep (128) -> MMA
+  B_TB_FULL = 12,    // prep (128) -> MMA
+  B_P_FULL = 13,     // prep (128) -> MMA
+  B_W_FULL = 14,     // MMA -> prep
+  B_MW_FULL = 15,    // prep (128) -> MMA
+  B_H0_FULL = 16,    // state (256) -> MMA
+  B_DMMA_FULL = 17,  // MMA -> state
+  B_D_FULL = 18,     // state (256) -> MMA
+  B_DU_EMPTY = 19,   // state (256) -> MMA
+  B_H_FULL = 20,     // MMA -> state, prep
+  NUM_BARS = 21
+};
+
 __device__ __forceinline__ void st_row_chunk(uint32_t tile, int row, int chunk, const float *v) {
   tc::st_shared_v4(tile + tc::sw128_off(row, chunk), tc::pack_bf16(v[0], v[1]),
                    tc::pack_bf16(v[2], v[3]), tc::pack_bf16(v[4], v[5]),
                    tc::pack_bf16(v[6], v[7]));
 }
-
-// Same, as the bf16 pair hi = bf16(x), lo = bf16(x - hi) into two tiles.
 __device__ __forceinline__ void st_row_chunk_split(uint32_t tile_hi, uint32_t tile_lo, int row,
                                                    int chunk, const float *v) {
   float hi[8], lo[8];
@@ -105,6 +125,13 @@ __device__ __forceinline__ void st_row_chunk_split(uint32_t tile_hi, uint32_t ti
   st_row_chunk(tile_lo, row, chunk, lo);
 }
 
+// Every lane has finished its shared/tensor-memory work for this hand-off (and fenced it);
+// one elected lane per warp then arrives.
+__device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
+  __syncwarp();
+  if (lane == 0) tc::mbar_arrive(bar);
+}
+
 template <bool OUT_F32>
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -114,358 +141,458 @@ __global__ void __launch_bounds__(NT, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = tc::smem_u32(smem);
-  float *bs2 = reinterpret_cast<float *>(smem + OFF_SMALL);  // b * log2(e)
-  float *betas = bs2 + 64;
-  float *gam = betas + 64;   // e^{b_r}
-  float *dtil = gam + 64;    // e^{b_C - b_r}
-  uint64_t *bars = reinterpret_cast<uint64_t *>(dtil + 64);  // full0, full1, mma
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 3);
+  float *gates = reinterpret_cast<float *>(smem + OFF_GATES);  // slot s: gates + 256 s
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BARS);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  float *Lf = reinterpret_cast<float *>(smem + OFF_L);  // [64][65]
-  float *Tf = reinterpret_cast<float *>(smem + OFF_T);  // [64][64]
-  float *Xf = reinterpret_cast<float *>(smem + OFF_X);  // merge scratch
-  const uint32_t bar_full[2] = {tc::smem_u32(&bars[0]), tc::smem_u32(&bars[1])};
-  const uint32_t bar_mma = tc::smem_u32(&bars[2]);
+  auto bar = [&](int i) { return tc::smem_u32(&bars[i]); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int wg = warp >> 2, q4 = warp & 3;
-  const int row = 32 * q4 + lane;  // the TMEM lane (accumulator row) this thread reads
+  const int row = 32 * q4 + lane;                        // TMEM lane this thread reads
   const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
 
   const int unit = blockIdx.x, n = unit / a.Hv, h = unit % a.Hv;
   const int hq = h / (a.Hv / a.Hqk);
   int batch, bos, eos;
   if (!seq_bounds(a.cu_seqlens, n, a.n_seqs, a.T, batch, bos, eos)) return;  // CTA-uniform
-  const float scale = a.scale;
+  const int nchunks = (eos - bos + C - 1) / C;
+  const int zbase = batch * a.T;
   const size_t st_off = ((size_t)n * a.Hv + h) * DK * DV;
 
   if (tid == 0) {
-    tc::mbar_init(bar_full[0], 1);
-    tc::mbar_init(bar_full[1], 1);
-    tc::mbar_init(bar_mma, 1);
+    // arrival counts: 1 = one thread (TMA expect_tx or tcgen05.commit), else one elected
+    // lane per warp of the signalling group (gates 1, prep 4, state 8, prep + state 12)
+    static constexpr uint16_t counts[NUM_BARS] = {1, 1, 1, 1, 1, 1, 1, 1, 12, 12, 1,
+                                                  4, 4, 4, 1, 4, 8, 1, 8, 8, 1};
+    for (int i = 0; i < NUM_BARS; ++i) tc::mbar_init(bar(i), counts[i]);
     *abort_flag = 0;
     tc::fence_barrier_init();
-    tc::prefetch_tmap(&tm_q);
-    tc::prefetch_tmap(&tm_k);
-    tc::prefetch_tmap(&tm_v);
   }
   if (warp == 0) {
     tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
     tc::tmem_relinquish();
   }
-
-  // Master state: this thread owns H[i][row] for i in [64 wg, 64 wg + 64).
-  float Hr[64];
-#pragma unroll
-  for (int m = 0; m < 64; ++m)
-    Hr[m] = a.state_in ? a.state_in[st_off + (size_t)(64 * wg + m) * DV + row] : 0.f;
-  auto write_shadow = [&]() {
-    const uint32_t tile = sb + OFF_H + (uint32_t)wg * 16384u;
-#pragma unroll
-    for (int cc = 0; cc < 8; ++cc) st_row_chunk(tile, row, cc, &Hr[8 * cc]);
-  };
-  write_shadow();
-  tc::fence_async_smem();
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  auto wait = [&](int i, uint32_t parity) { tc::mbar_wait(bar(i), parity, abort_flag); };
 
-  const int nchunks = (eos - bos + C - 1) / C;
-  const int zbase = batch * a.T;  // token row of (batch, t = 0) in the [B*T] axis
-  auto issue_tma = [&](int stage, int t0) {
-    const uint32_t dst = sb + (uint32_t)stage * STAGE_BYTES;
-    const int z = zbase + t0;
-    tc::mbar_arrive_expect_tx(bar_full[stage], STAGE_BYTES);
-    tc::tma_load_3d(dst + OFF_K0, &tm_k, bar_full[stage], 0, hq, z);
-    tc::tma_load_3d(dst + OFF_K1, &tm_k, bar_full[stage], 64, hq, z);
-    tc::tma_load_3d(dst + OFF_Q0, &tm_q, bar_full[stage], 0, hq, z);
-    tc::tma_load_3d(dst + OFF_Q1, &tm_q, bar_full[stage], 64, hq, z);
-    tc::tma_load_3d(dst + OFF_V0, &tm_v, bar_full[stage], 0, h, z);
-    tc::tma_load_3d(dst + OFF_V1, &tm_v, bar_full[stage], 64, h, z);
-  };
-  int tma_issued = 0;  // chunks whose loads have been issued (thread 0 only)
-  if (tid == 0 && nchunks > 0) {
-    issue_tma(0, bos);
-    tma_issued = 1;
-  }
-  uint32_t mma_phase = 0;
-  auto mma_wait = [&]() {
-    tc::mbar_wait(bar_mma, mma_phase, abort_flag);
-    mma_phase ^= 1u;
-    tc::tc_fence_after();
-  };
-  auto sync_for_mma = [&]() {  // smem writes + TMEM reads done -> next MMA may run
-    tc::fence_async_smem();
-    tc::tc_fence_before();
-    __syncthreads();
-  };
-
-  // gates / write strengths of the next chunk are loaded one chunk ahead (warp 0)
-  float gn0 = 0.f, gn1 = 0.f, bn0 = 0.f, bn1 = 0.f;
-  auto load_gb = [&](int t0) {
-    const int L = min(C, eos - t0);
-    const size_t i0 = ((size_t)zbase + t0 + lane) * a.Hv + h;
-    gn0 = gn1 = bn0 = bn1 = 0.f;
-    if (lane < L) {
-      gn0 = a.g ? a.g[i0] : 0.f;
-      bn0 = a.beta[i0];
-    }
-    if (lane + 32 < L) {
-      gn1 = a.g ? a.g[i0 + (size_t)32 * a.Hv] : 0.f;
-      bn1 = a.beta[i0 + (size_t)32 * a.Hv];
-    }
-  };
-  if (warp == 0 && nchunks > 0) load_gb(bos);
-
-  for (int c = 0; c < nchunks; ++c) {
-    const int t0 = bos + c * C;
-    const int L = min(C, eos - t0);
-    const int s = c & 1;
-    const uint32_t stg = sb + (uint32_t)s * STAGE_BYTES;
-
-    // ---- cumulative log decay of this chunk (rows past the end have g = beta = 0) ----
-    if (warp == 0) {
-      float g0 = gn0, g1 = gn1;
-      const float b0 = bn0, b1 = bn1;
-      if (c + 1 < nchunks) load_gb(t0 + C);
+  if (wg == 0) {
+    // =========================================================== producer roles
+    if (warp == 0 && lane == 0 && nchunks > 0) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1, z = zbase + bos + c * C;
+        const uint32_t dst = sb + OFF_QK + (uint32_t)s * QK_BYTES;
+        if (c >= 2) wait(B_QK_EMPTY + s, (((uint32_t)c >> 1) & 1u) ^ 1u);
+        if (*abort_flag) break;
+        tc::mbar_arrive_expect_tx(bar(B_QK_FULL + s), QK_BYTES);
+        tc::tma_load_3d(dst + QK_K0, &tm_k, bar(B_QK_FULL + s), 0, hq, z);
+        tc::tma_load_3d(dst + QK_K1, &tm_k, bar(B_QK_FULL + s), 64, hq, z);
+        tc::tma_load_3d(dst + QK_Q0, &tm_q, bar(B_QK_FULL + s), 0, hq, z);
+        tc::tma_load_3d(dst + QK_Q1, &tm_q, bar(B_QK_FULL + s), 64, hq, z);
+        if (c >= 1) wait(B_V_EMPTY, (uint32_t)(c - 1) & 1u);
+        if (*abort_flag) break;
+        tc::mbar_arrive_expect_tx(bar(B_V_FULL), V_BYTES);
+        tc::tma_load_3d(sb + OFF_V, &tm_v, bar(B_V_FULL), 0, h, z);
+        tc::tma_load_3d(sb + OFF_V + 8192, &tm_v, bar(B_V_FULL), 64, h, z);
+      }
+    } else if (warp == 1 && lane == 0 && nchunks > 0) {
+      // ------------------------------------------------------- MMA issuer
+      auto issue_G = [&](int c) {
+        const int s = c & 1;
+        wait(B_QK_FULL + s, ((uint32_t)c >> 1) & 1u);
+        if (c > 0) wait(B_G_EMPTY, (uint32_t)(c - 1) & 1u);
+        if (*abort_flag) return;
+        tc::tc_fence_after();
+        const uint32_t stg = sb + OFF_QK + (uint32_t)s * QK_BYTES;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float y0 = __shfl_up_sync(0xffffffffu, g0, off);
-        const float y1 = __shfl_up_sync(0xffffffffu, g1, off);
-        if (lane >= off) {
-          g0 += y0;
-          g1 += y1;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t d = tc::sdesc_sw128(stg + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024);
+          tc::mma_bf16(tmem + COL_G, d, d, ID_G, kk > 0);
         }
-      }
-      g1 += __shfl_sync(0xffffffffu, g0, 31);
-      const float blast = __shfl_sync(0xffffffffu, g1, 31);
-      bs2[lane] = g0 * LOG2E;
-      bs2[lane + 32] = g1 * LOG2E;
-      betas[lane] = b0;
-      betas[lane + 32] = b1;
-      gam[lane] = exp2f(g0 * LOG2E);
-      gam[lane + 32] = exp2f(g1 * LOG2E);
-      dtil[lane] = exp2f((blast - g0) * LOG2E);
-      dtil[lane + 32] = exp2f((blast - g1) * LOG2E);
-    }
-    if (tid == 0 && c + 1 < nchunks) {
-      issue_tma(s ^ 1, t0 + C);
-      ++tma_issued;
-    }
-    tc::mbar_wait(bar_full[s], (uint32_t)(c >> 1) & 1u, abort_flag);
-    __syncthreads();
-
-    // ---- G = [K; Q] K^T  (M=128, N=64, K=128) ----
-    if (tid == 0 && !*abort_flag) {
-      tc::tc_fence_after();
+        tc::mma_commit(bar(B_G_FULL));
+      };
+      auto issue_WU = [&](int c) {
+        wait(B_TB_FULL, (uint32_t)c & 1u);
+        wait(B_V_FULL, (uint32_t)c & 1u);
+        if (c > 0) wait(B_DU_EMPTY, (uint32_t)(c - 1) & 1u);
+        if (*abort_flag) return;
+        tc::tc_fence_after();
+        const uint32_t stg = sb + OFF_QK + (uint32_t)(c & 1) * QK_BYTES;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t at = stg + (kk >> 2) * 16384u + (kk & 3) * 32u;
-        const uint64_t d = tc::sdesc_sw128(at, 16, 1024);
-        tc::mma_bf16(tmem + COL_G, d, d, ID_G, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ak = tc::sdesc_sw128(stg + QK_K0 + kk * 2048u, 16384, 1024);
+          const uint64_t av = tc::sdesc_sw128(sb + OFF_V + kk * 2048u, 8192, 1024);
+          tc::mma_bf16(tmem + COL_W, ak, tc::sdesc_sw128(sb + OFF_RX + kk * 32u, 16, 1024), ID_MNK, kk > 0);
+          tc::mma_bf16(tmem + COL_W, ak, tc::sdesc_sw128(sb + OFF_RX + 8192 + kk * 32u, 16, 1024), ID_MNK, 1);
+          tc::mma_bf16(tmem + COL_DU, av, tc::sdesc_sw128(sb + OFF_RL + kk * 32u, 16, 1024), ID_MNK, kk > 0);
+          tc::mma_bf16(tmem + COL_DU, av, tc::sdesc_sw128(sb + OFF_RL + 8192 + kk * 32u, 16, 1024), ID_MNK, 1);
+        }
+        tc::mma_commit(bar(B_W_FULL));
+        tc::mma_commit(bar(B_V_EMPTY));
+      };
+      auto issue_DO = [&](int c) {
+        wait(B_MW_FULL, (uint32_t)c & 1u);
+        wait(B_H0_FULL, (uint32_t)c & 1u);
+        if (*abort_flag) return;
+        tc::tc_fence_after();
+        const uint32_t stg = sb + OFF_QK + (uint32_t)(c & 1) * QK_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bw = tc::sdesc_sw128(sb + OFF_RT + kk * 2048u, 8192, 1024);
+          tc::mma_bf16_ta(tmem + COL_DU, tmem + COL_H0 + 8 * kk, bw, ID_KMN64, 1);
+        }
+        tc::mma_commit(bar(B_DMMA_FULL));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bq =
+              tc::sdesc_sw128(stg + QK_Q0 + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024);
+          tc::mma_bf16_ta(tmem + COL_OA, tmem + COL_H0 + 8 * kk, bq, ID_KK64, kk > 0);
+        }
+      };
+      auto issue_HO = [&](int c) {
+        wait(B_D_FULL, (uint32_t)c & 1u);
+        wait(B_P_FULL, (uint32_t)c & 1u);
+        if (*abort_flag) return;
+        tc::tc_fence_after();
+        const uint32_t stg = sb + OFF_QK + (uint32_t)(c & 1) * QK_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bk = tc::sdesc_sw128(stg + QK_K0 + kk * 2048u, 16384, 1024);
+          tc::mma_bf16(tmem + COL_HU, tc::sdesc_sw128(sb + OFF_DTH + kk * 32u, 16, 1024), bk, ID_KMN128, kk > 0);
+          tc::mma_bf16(tmem + COL_HU, tc::sdesc_sw128(sb + OFF_DTL + kk * 32u, 16, 1024), bk, ID_KMN128, 1);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t adh = tc::sdesc_sw128(sb + OFF_DH + kk * 32u, 16, 1024);
+          const uint64_t adl = tc::sdesc_sw128(sb + OFF_DL + kk * 32u, 16, 1024);
+          const uint64_t bph = tc::sdesc_sw128(sb + OFF_P + kk * 32u, 16, 1024);
+          const uint64_t bpl = tc::sdesc_sw128(sb + OFF_P + 8192 + kk * 32u, 16, 1024);
+          tc::mma_bf16(tmem + COL_OB, adh, bph, ID_KK64, kk > 0);
+          tc::mma_bf16(tmem + COL_OB, adl, bph, ID_KK64, 1);
+          tc::mma_bf16(tmem + COL_OB, adh, bpl, ID_KK64, 1);
+        }
+        tc::mma_commit(bar(B_H_FULL));
+        tc::mma_commit(bar(B_QK_EMPTY + (c & 1)));
+      };
+      issue_G(0);
+      issue_WU(0);
+      for (int c = 0; c < nchunks; ++c) {
+        issue_DO(c);
+        if (c + 1 < nchunks) issue_G(c + 1);
+        issue_HO(c);
+        if (c + 1 < nchunks) issue_WU(c + 1);
       }
-      tc::mma_commit(bar_mma);
+    } else if (warp == 2) {
+      // ------------------------------------------------------- gates
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c & 1, t0 = bos + c * C, L = min(C, eos - t0);
+        if (c >= 2) wait(B_GATE_EMPTY + s, ((uint32_t)(c - 2) >> 1) & 1u);
+        float g0 = 0.f, g1 = 0.f, b0 = 0.f, b1 = 0.f;
+        const size_t i0 = ((size_t)zbase + t0 + lane) * a.Hv + h;
+        if (lane < L) {
+          g0 = a.g ? a.g[i0] : 0.f;
+          b0 = a.beta[i0];
+        }
+        if (lane + 32 < L) {
+          g1 = a.g ? a.g[i0 + (size_t)32 * a.Hv] : 0.f;
+          b1 = a.beta[i0 + (size_t)32 * a.Hv];
+        }
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y0 = __shfl_up_sync(0xffffffffu, g0, off);
+          const float y1 = __shfl_up_sync(0xffffffffu, g1, off);
+          if (lane >= off) {
+            g0 += y0;
+            g1 += y1;
+          }
+        }
+        g1 += __shfl_sync(0xffffffffu, g0, 31);
+        const float blast = __shfl_sync(0xffffffffu, g1, 31);
+        float *gs = gates + 256 * s;  // bs2[64], beta[64], gam[64], dtil[64]
+        gs[lane] = g0 * LOG2E;
+        gs[lane + 32] = g1 * LOG2E;
+        gs[64 + lane] = b0;
+        gs[96 + lane] = b1;
+        gs[128 + lane] = exp2f(g0 * LOG2E);
+        gs[160 + lane] = exp2f(g1 * LOG2E);
+        gs[192 + lane] = exp2f((blast - g0) * LOG2E);
+        gs[224 + lane] = exp2f((blast - g1) * LOG2E);
+        warp_arrive(bar(B_GATE_FULL + s), lane);
+      }
     }
-    mma_wait();
-    {
-      float v[32];
-      tc::tmem_ld32(tmem + lane_off + COL_G + 32 * wg, v);
-      if (row < 64) {  // L row r: beta_r Gamma_rs (k_r . k_s), s < r
+  } else if (wg == 1) {
+    // =========================================================== prep (chunk c+1 ahead)
+    const int pt = tid - 128;  // 0..127
+    float *LT = reinterpret_cast<float *>(smem + OFF_RL);  // L^T fp32 [64 s][64 r]
+    float *Tf = reinterpret_cast<float *>(smem + OFF_RT);  // T fp32 [64][64], row-major
+    float *Xs = reinterpret_cast<float *>(smem + OFF_RX);  // merge scratch: 3 x [16][16]
+    float *TDT = Xs + 3 * 256;                             // diagonal blocks transposed [4][16 m][16 r]
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      const float *gs = gates + 256 * s;
+      wait(B_GATE_FULL + s, ((uint32_t)c >> 1) & 1u);
+      wait(B_G_FULL, (uint32_t)c & 1u);
+      tc::tc_fence_after();
+      // ---- L^T (TMEM lanes 0-63 hold rows r of K K^T): L_rs = beta_r Gamma_rs (k_r . k_s), s < r ----
+      if (q4 < 2) {
         const int r = row;
-        const float br = bs2[r], bt = betas[r];
+        const float br = gs[r], bt = gs[64 + r];
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc) {
-          const int s_ = 32 * wg + cc;
-          Lf[r * 65 + s_] = (s_ < r) ? bt * exp2f(br - bs2[s_]) * v[cc] : 0.f;
+        for (int half = 0; half < 2; ++half) {
+          float v[32], bs[32];
+          tc::tmem_ld32(tmem + lane_off + COL_G + 32 * half, v);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 b4 = reinterpret_cast<const float4 *>(gs)[8 * half + q];
+            bs[4 * q] = b4.x; bs[4 * q + 1] = b4.y; bs[4 * q + 2] = b4.z; bs[4 * q + 3] = b4.w;
+          }
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc) {
+            const int s_ = 32 * half + cc;
+            LT[s_ * 64 + r] = (s_ < r) ? bt * exp2f(br - bs[cc]) * v[cc] : 0.f;
+          }
         }
-      } else {  // P row r: scale Gamma_rs (q_r . k_s), s <= r  -> bf16, K-major B tile
-        const int r = row - 64;
-        const float br = bs2[r];
+      }
+      tc::named_bar(1, 128);
+      // ---- T = (I + L)^-1, diagonal 16x16 blocks by forward substitution (one column each) ----
+      if (pt < 64) {
+        const int blk = pt >> 4, cI = pt & 15, R = 16 * blk;
+        float x[16];
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc) {
-          const int s_ = 32 * wg + cc;
-          v[cc] = (s_ <= r) ? scale * exp2f(br - bs2[s_]) * v[cc] : 0.f;
+        for (int r = 0; r < 16; ++r) x[r] = (r == cI) ? 1.f : 0.f;
+#pragma unroll
+        for (int r = 1; r < 16; ++r) {
+          float acc = 0.f;
+#pragma unroll
+          for (int q = 0; q < r; ++q) acc += LT[(R + q) * 64 + R + r] * x[q];
+          if (r > cI) x[r] = -acc;
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) st_row_chunk_split(sb + OFF_P_H, sb + OFF_P_L, r, 4 * wg + q, &v[8 * q]);
+        for (int r = 0; r < 16; ++r) {
+          Tf[(R + r) * 64 + R + cI] = x[r];
+          TDT[blk * 256 + cI * 16 + r] = x[r];  // (T_bb)^T[m = cI][r]
+        }
       }
-    }
-    tc::tc_fence_before();
-    __syncthreads();
-
-    // ---- T = (I + L)^-1: 16x16 diagonal blocks by forward substitution ----
-    if (tid < 64) {
-      const int blk = tid >> 4, cI = tid & 15, R = 16 * blk;
-      float x[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) x[r] = (r == cI) ? 1.f : 0.f;
-#pragma unroll
-      for (int r = 1; r < 16; ++r) {
-        float acc = 0.f;
-#pragma unroll
-        for (int q = 0; q < r; ++q) acc += Lf[(R + r) * 65 + R + q] * x[q];
-        if (r > cI) x[r] = -acc;
-      }
-#pragma unroll
-      for (int r = 0; r < 16; ++r) Tf[(R + r) * 64 + R + cI] = x[r];
-    }
-    __syncthreads();
-    // ---- block merges: T_ij = -T_ii sum_{k=j}^{i-1} L_ik T_kj, by distance d = i - j ----
+      tc::named_bar(1, 128);
+      // ---- block merges by distance d = i - j:  X = sum_{k=j}^{i-1} L_ik T_kj,  T_ij = -T_ii X.
+      //      4x4 register tiles, the K range split over ks adjacent lanes (shuffle-reduced). ----
 #pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-      const int nblk = 4 - d;
-      for (int e = tid; e < nblk * 256; e += NT) {  // X = sum_k L_ik T_kj
-        const int bi = e >> 8, rc = e & 255, r = rc >> 4, cI = rc & 15;
-        const int i = bi + d, j = bi;
-        float acc = 0.f;
-        for (int k = j; k < i; ++k) {
+      for (int d = 1; d < 4; ++d) {
+        const int nb = 4 - d;                   // blocks in this round
+        const int ks = d == 1 ? 2 : (d == 2 ? 4 : 8);
+        const int item = pt, part = item & (ks - 1), tile = item / ks;
+        const bool active = tile < nb * 16;
+        const int blk = tile >> 4, tr = (tile >> 2) & 3, tcI = tile & 3;
+        const int i = blk + d, j = blk;
+        float acc[16];
 #pragma unroll
-          for (int m = 0; m < 16; ++m)
-            acc += Lf[(16 * i + r) * 65 + 16 * k + m] * Tf[(16 * k + m) * 64 + 16 * j + cI];
+        for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+        if (active) {
+          const int kn = 16 * d / ks, k0 = 16 * j + part * kn;
+          const int r0 = 16 * i + 4 * tr, c0 = 16 * j + 4 * tcI;
+          for (int m = 0; m < kn; ++m) {
+            const float4 l4 = *reinterpret_cast<const float4 *>(&LT[(k0 + m) * 64 + r0]);
+            const float4 t4 = *reinterpret_cast<const float4 *>(&Tf[(k0 + m) * 64 + c0]);
+            const float la[4] = {l4.x, l4.y, l4.z, l4.w}, ta[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+            for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+              for (int b2 = 0; b2 < 4; ++b2) acc[4 * a2 + b2] += la[a2] * ta[b2];
+          }
         }
-        Xf[e] = acc;
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1)
+          if (off < ks)
+#pragma unroll
+            for (int t = 0; t < 16; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+        if (active && part == 0) {
+#pragma unroll
+          for (int a2 = 0; a2 < 4; ++a2)
+            *reinterpret_cast<float4 *>(&Xs[blk * 256 + (4 * tr + a2) * 16 + 4 * tcI]) =
+                make_float4(acc[4 * a2], acc[4 * a2 + 1], acc[4 * a2 + 2], acc[4 * a2 + 3]);
+        }
+        tc::named_bar(1, 128);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+        if (active) {  // T_ij = -T_ii X  (K = 16 split over ks lanes)
+          const int kn = 16 / ks, m0 = part * kn;
+#pragma unroll 1
+          for (int m = m0; m < m0 + kn; ++m) {
+            const float4 l4 = *reinterpret_cast<const float4 *>(&TDT[i * 256 + m * 16 + 4 * tr]);
+            const float4 x4 = *reinterpret_cast<const float4 *>(&Xs[blk * 256 + m * 16 + 4 * tcI]);
+            const float la[4] = {l4.x, l4.y, l4.z, l4.w}, xa[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+            for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+              for (int b2 = 0; b2 < 4; ++b2) acc[4 * a2 + b2] += la[a2] * xa[b2];
+          }
+        }
+#pragma unroll
+        for (int off = 1; off < 8; off <<= 1)
+          if (off < ks)
+#pragma unroll
+            for (int t = 0; t < 16; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+        if (active && part == 0) {
+#pragma unroll
+          for (int a2 = 0; a2 < 4; ++a2)
+            *reinterpret_cast<float4 *>(&Tf[(16 * i + 4 * tr + a2) * 64 + 16 * j + 4 * tcI]) =
+                make_float4(-acc[4 * a2], -acc[4 * a2 + 1], -acc[4 * a2 + 2], -acc[4 * a2 + 3]);
+        }
+        tc::named_bar(1, 128);
       }
-      __syncthreads();
-      for (int e = tid; e < nblk * 256; e += NT) {  // T_ij = -T_ii X
-        const int bi = e >> 8, rc = e & 255, r = rc >> 4, cI = rc & 15;
-        const int i = bi + d, j = bi;
-        float acc = 0.f;
+      // ---- T diag(beta) (over L's region) and T diag(beta gamma) (over the scratch) ----
+      for (int e = pt; e < 64 * 8; e += 128) {
+        const int r = e >> 3, q = e & 7;
+        float tb[8], tbg[8];
+        const float4 ta = *reinterpret_cast<const float4 *>(&Tf[r * 64 + 8 * q]);
+        const float4 tb4 = *reinterpret_cast<const float4 *>(&Tf[r * 64 + 8 * q + 4]);
+        const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb4.x, tb4.y, tb4.z, tb4.w};
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
-          acc += Tf[(16 * i + r) * 64 + 16 * i + m] * Xf[(bi << 8) + m * 16 + cI];
-        Tf[(16 * i + r) * 64 + 16 * j + cI] = -acc;
+        for (int m = 0; m < 8; ++m) {
+          const int s_ = 8 * q + m;
+          tb[m] = (s_ <= r) ? tv[m] * gs[64 + s_] : 0.f;
+          tbg[m] = tb[m] * gs[128 + s_];
+        }
+        st_row_chunk_split(sb + OFF_RL, sb + OFF_RL + 8192, r, q, tb);
+        st_row_chunk_split(sb + OFF_RX, sb + OFF_RX + 8192, r, q, tbg);
       }
-      __syncthreads();
-    }
-    // ---- T diag(beta) and T diag(beta gamma) as bf16 hi/lo K-major B tiles ----
-    for (int e = tid; e < 64 * 8; e += NT) {
-      const int r = e >> 3, q = e & 7;
-      float tb[8], tbg[8];
+      tc::fence_async_smem();
+      warp_arrive(bar(B_TB_FULL), lane);
+      // ---- P rows (TMEM lanes 64-127): scale Gamma_rs (q_r . k_s), s <= r ----
+      if (c > 0) wait(B_H_FULL, (uint32_t)(c - 1) & 1u);  // Ob(c-1) has read P
+      if (q4 >= 2) {
+        const int r = row - 64;
+        const float br = gs[r];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int s_ = 8 * q + m;
-        const float t = (s_ <= r) ? Tf[r * 64 + s_] : 0.f;
-        tb[m] = t * betas[s_];
-        tbg[m] = tb[m] * gam[s_];
-      }
-      st_row_chunk_split(sb + OFF_TB_H, sb + OFF_TB_L, r, q, tb);
-      st_row_chunk_split(sb + OFF_TBG_H, sb + OFF_TBG_L, r, q, tbg);
-    }
-    sync_for_mma();
-
-    // ---- W^T = K^T (T diag(beta gamma))^T,  U^T = V^T (T diag(beta))^T  (M=128, N=64, K=64) ----
-    if (tid == 0 && !*abort_flag) {
-      tc::tc_fence_after();
+        for (int half = 0; half < 2; ++half) {
+          float v[32];
+          tc::tmem_ld32(tmem + lane_off + COL_G + 32 * half, v);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ak = tc::sdesc_sw128(stg + OFF_K0 + kk * 2048u, 16384, 1024);
-        const uint64_t av = tc::sdesc_sw128(stg + OFF_V0 + kk * 2048u, 8192, 1024);
-        tc::mma_bf16(tmem + COL_W, ak, tc::sdesc_sw128(sb + OFF_TBG_H + kk * 32u, 16, 1024), ID_MNK, kk > 0);
-        tc::mma_bf16(tmem + COL_W, ak, tc::sdesc_sw128(sb + OFF_TBG_L + kk * 32u, 16, 1024), ID_MNK, 1);
-        tc::mma_bf16(tmem + COL_DU, av, tc::sdesc_sw128(sb + OFF_TB_H + kk * 32u, 16, 1024), ID_MNK, kk > 0);
-        tc::mma_bf16(tmem + COL_DU, av, tc::sdesc_sw128(sb + OFF_TB_L + kk * 32u, 16, 1024), ID_MNK, 1);
-      }
-      tc::mma_commit(bar_mma);
-    }
-    mma_wait();
-    {  // -W^T -> bf16 (row i = TMEM lane, 64 values of r: MN-major B for the Delta product)
-      float v[32];
-      tc::tmem_ld32(tmem + lane_off + COL_W + 32 * wg, v);
+          for (int cc = 0; cc < 32; ++cc) {
+            const int s_ = 32 * half + cc;
+            v[cc] = (s_ <= r) ? a.scale * exp2f(br - gs[s_]) * v[cc] : 0.f;
+          }
 #pragma unroll
-      for (int cc = 0; cc < 32; ++cc) v[cc] = -v[cc];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) st_row_chunk(sb + OFF_W, row, 4 * wg + q, &v[8 * q]);
-    }
-    sync_for_mma();
-
-    // ---- Delta^T = U^T + H0^T (-W^T) (K=128, onto U^T);  Oa = H0^T Q^T ----
-    if (tid == 0 && !*abort_flag) {
-      tc::tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t ah = tc::sdesc_sw128(sb + OFF_H + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024);
-        const uint64_t bw = tc::sdesc_sw128(sb + OFF_W + kk * 2048u, 8192, 1024);
-        const uint64_t bq = tc::sdesc_sw128(stg + OFF_Q0 + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024);
-        tc::mma_bf16(tmem + COL_DU, ah, bw, ID_KMN64, 1);
-        tc::mma_bf16(tmem + COL_OA, ah, bq, ID_KK64, kk > 0);
-      }
-      tc::mma_commit(bar_mma);
-    }
-    mma_wait();
-    {  // Delta^T and Delta~^T (scaled by e^{b_C - b_s}) -> bf16 hi/lo K-major A tiles
-      float v[32], w[32];
-      tc::tmem_ld32(tmem + lane_off + COL_DU + 32 * wg, v);
-#pragma unroll
-      for (int cc = 0; cc < 32; ++cc) w[cc] = v[cc] * dtil[32 * wg + cc];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        st_row_chunk_split(sb + OFF_D_H, sb + OFF_D_L, row, 4 * wg + q, &v[8 * q]);
-        st_row_chunk_split(sb + OFF_DT_H, sb + OFF_DT_L, row, 4 * wg + q, &w[8 * q]);
-      }
-    }
-    sync_for_mma();
-
-    // ---- Ob = Delta^T P^T (N=64, K=64);  Hupd = Delta~^T K (N=128, K=64); hi/lo pairs ----
-    if (tid == 0 && !*abort_flag) {
-      tc::tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t adh = tc::sdesc_sw128(sb + OFF_D_H + kk * 32u, 16, 1024);
-        const uint64_t adl = tc::sdesc_sw128(sb + OFF_D_L + kk * 32u, 16, 1024);
-        const uint64_t bph = tc::sdesc_sw128(sb + OFF_P_H + kk * 32u, 16, 1024);
-        const uint64_t bpl = tc::sdesc_sw128(sb + OFF_P_L + kk * 32u, 16, 1024);
-        const uint64_t bk = tc::sdesc_sw128(stg + OFF_K0 + kk * 2048u, 16384, 1024);
-        tc::mma_bf16(tmem + COL_OB, adh, bph, ID_KK64, kk > 0);
-        tc::mma_bf16(tmem + COL_OB, adl, bph, ID_KK64, 1);
-        tc::mma_bf16(tmem + COL_OB, adh, bpl, ID_KK64, 1);
-        tc::mma_bf16(tmem + COL_HU, tc::sdesc_sw128(sb + OFF_DT_H + kk * 32u, 16, 1024), bk, ID_KMN128, kk > 0);
-        tc::mma_bf16(tmem + COL_HU, tc::sdesc_sw128(sb + OFF_DT_L + kk * 32u, 16, 1024), bk, ID_KMN128, 1);
-      }
-      tc::mma_commit(bar_mma);
-    }
-    mma_wait();
-    {  // outputs: O[r][j] = scale gamma_r Oa[j][r] + Ob[j][r]
-      float oa[32], ob[32];
-      tc::tmem_ld32(tmem + lane_off + COL_OA + 32 * wg, oa);
-      tc::tmem_ld32(tmem + lane_off + COL_OB + 32 * wg, ob);
-      const size_t obase = ((size_t)zbase + t0) * a.Hv + h;
-#pragma unroll
-      for (int cc = 0; cc < 32; ++cc) {
-        const int r = 32 * wg + cc;
-        if (r < L) {
-          const float val = scale * gam[r] * oa[cc] + ob[cc];
-          const size_t off = (obase + (size_t)r * a.Hv) * DV + row;
-          if constexpr (OUT_F32)
-            static_cast<float *>(a.o)[off] = val;
-          else
-            static_cast<__nv_bfloat16 *>(a.o)[off] = __float2bfloat16_rn(val);
+          for (int q = 0; q < 4; ++q)
+            st_row_chunk_split(sb + OFF_P, sb + OFF_P + 8192, r, 4 * half + q, &v[8 * q]);
         }
       }
-    }
-    {  // state: H = gamma_C H + Hupd; refresh the bf16 shadow
-      const float gC = gam[63];
+      tc::fence_async_smem();
+      tc::tc_fence_before();
+      warp_arrive(bar(B_P_FULL), lane);
+      warp_arrive(bar(B_G_EMPTY), lane);
+      // ---- -W^T (TMEM lane i, 64 values of r) -> MN-major B tile over T's region ----
+      wait(B_W_FULL, (uint32_t)c & 1u);
+      tc::tc_fence_after();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        float u[32];
-        tc::tmem_ld32(tmem + lane_off + COL_HU + 64 * wg + 32 * half, u);
+        float v[32];
+        tc::tmem_ld32(tmem + lane_off + COL_W + 32 * half, v);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) Hr[32 * half + m] = gC * Hr[32 * half + m] + u[m];
+        for (int cc = 0; cc < 32; ++cc) v[cc] = -v[cc];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) st_row_chunk(sb + OFF_RT, row, 4 * half + q, &v[8 * q]);
       }
-      write_shadow();
+      tc::fence_async_smem();
+      tc::tc_fence_before();
+      warp_arrive(bar(B_MW_FULL), lane);
+      warp_arrive(bar(B_GATE_EMPTY + s), lane);
     }
-    sync_for_mma();
-    tc::tc_fence_after();
+  } else {
+    // =========================================================== state chain
+    const int swg = wg - 2;  // 0 or 1: key rows [64 swg, 64 swg + 64), value-column halves
+    float Hr[64];
+#pragma unroll
+    for (int m = 0; m < 64; ++m)
+      Hr[m] = a.state_in ? a.state_in[st_off + (size_t)(64 * swg + m) * DV + row] : 0.f;
+    auto store_h0 = [&]() {  // H0^T row j (this lane), k = key rows of this half, bf16 pairs
+      uint32_t pk[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) pk[t] = tc::pack_bf16(Hr[2 * t], Hr[2 * t + 1]);
+      tc::tmem_st32(tmem + lane_off + COL_H0 + 32 * swg, pk);
+      tc::tc_fence_before();
+    };
+    if (nchunks > 0) {
+      store_h0();
+      warp_arrive(bar(B_H0_FULL), lane);
+    }
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1, t0 = bos + c * C, L = min(C, eos - t0);
+      const float *gs = gates + 256 * s;
+      wait(B_GATE_FULL + s, ((uint32_t)c >> 1) & 1u);
+      wait(B_DMMA_FULL, (uint32_t)c & 1u);
+      tc::tc_fence_after();
+      // ---- Delta^T, Delta~^T -> bf16 hi/lo K-major A tiles (row j, columns r of this half) ----
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        float v[16], w[16];
+        const int r0 = 32 * swg + 16 * part;
+        tc::tmem_ld16(tmem + lane_off + COL_DU + r0, v);
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) w[cc] = v[cc] * gs[192 + r0 + cc];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int ch = (r0 >> 3) + q;
+          st_row_chunk_split(sb + OFF_DH, sb + OFF_DL, row, ch, &v[8 * q]);
+          st_row_chunk_split(sb + OFF_DTH, sb + OFF_DTL, row, ch, &w[8 * q]);
+        }
+      }
+      tc::fence_async_smem();
+      tc::tc_fence_before();
+      warp_arrive(bar(B_D_FULL), lane);
+      warp_arrive(bar(B_DU_EMPTY), lane);
+      wait(B_H_FULL, (uint32_t)c & 1u);
+      tc::tc_fence_after();
+      // ---- outputs: O[r][j] = scale gamma_r Oa[j][r] + Ob[j][r] ----
+      {
+        const size_t obase = ((size_t)zbase + t0) * a.Hv + h;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          float oa[16], ob[16];
+          const int r0 = 32 * swg + 16 * part;
+          tc::tmem_ld16(tmem + lane_off + COL_OA + r0, oa);
+          tc::tmem_ld16(tmem + lane_off + COL_OB + r0, ob);
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) {
+            const int r = r0 + cc;
+            if (r < L) {
+              const float val = a.scale * gs[128 + r] * oa[cc] + ob[cc];
+              const size_t off = (obase + (size_t)r * a.Hv) * DV + row;
+              if constexpr (OUT_F32)
+                static_cast<float *>(a.o)[off] = val;
+              else
+                static_cast<__nv_bfloat16 *>(a.o)[off] = __float2bfloat16_rn(val);
+            }
+          }
+        }
+      }
+      // ---- state: H = gamma_C H + Hupd; new H0^T operand ----
+      {
+        const float gC = gs[128 + 63];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float u[32];
+          tc::tmem_ld32(tmem + lane_off + COL_HU + 64 * swg + 32 * half, u);
+#pragma unroll
+          for (int m = 0; m < 32; ++m) Hr[32 * half + m] = gC * Hr[32 * half + m] + u[m];
+        }
+        store_h0();
+      }
+      warp_arrive(bar(B_H0_FULL), lane);
+      warp_arrive(bar(B_GATE_EMPTY + s), lane);
+    }
+    if (a.state_out) {
+#pragma unroll
+      for (int m = 0; m < 64; ++m) a.state_out[st_off + (size_t)(64 * swg + m) * DV + row] = Hr[m];
+    }
   }
 
-  if (a.state_out) {
-#pragma unroll
-    for (int m = 0; m < 64; ++m) a.state_out[st_off + (size_t)(64 * wg + m) * DV + row] = Hr[m];
-  }
-  // Wind down: make sure no TMA write into this CTA's shared memory is still in flight.
-  if (tid == 0 && *abort_flag) {
-    for (int c = 0; c < tma_issued; ++c) tc::mbar_wait(bar_full[c & 1], (uint32_t)(c >> 1) & 1u, abort_flag, 1u << 20);
-  }
   tc::tc_fence_before();
   __syncthreads();
   if (warp == 0) {
