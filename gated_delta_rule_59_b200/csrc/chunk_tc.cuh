@@ -44,6 +44,7 @@
 #include <cuda.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "chunk_simt.cuh"
 #include "tc_ptx.cuh"
@@ -113,6 +114,7 @@ __device__ __forceinline__ void st_row_chunk(uint32_t tile, int row, int chunk, 
                    tc::pack_bf16(v[2], v[3]), tc::pack_bf16(v[4], v[5]),
                    tc::pack_bf16(v[6], v[7]));
 }
+// Same, as the bf16 pair hi = bf16(x), lo = bf16(x - hi) into two tiles.
 __device__ __forceinline__ void st_row_chunk_split(uint32_t tile_hi, uint32_t tile_lo, int row,
                                                    int chunk, const float *v) {
   float hi[8], lo[8];
@@ -123,6 +125,83 @@ __device__ __forceinline__ void st_row_chunk_split(uint32_t tile_hi, uint32_t ti
   }
   st_row_chunk(tile_hi, row, chunk, hi);
   st_row_chunk(tile_lo, row, chunk, lo);
+}
+
+// One round of the block merges of T = (I + L)^-1 (blocks of 16; distance D = i - j):
+//   X_i = sum_{k=j}^{i-1} L_ik T_kj,   T_ij = -T_ii X_i   for the 4 - D blocks (i, i - D).
+// 128 threads; a thread owns a 4x4 tile of one block and 1/KS of the K range.
+template <int D>
+__device__ __forceinline__ void merge_round(int pt, const float *LT, float *Tf, float *Xs,
+                                            const float *TDT) {
+  constexpr int NB = 4 - D, KS = D == 1 ? 2 : (D == 2 ? 4 : 8);
+  constexpr int KN = 16 * D / KS, KN2 = 16 / KS;
+  const int part = pt & (KS - 1), tile = pt / KS;
+  const bool active = tile < NB * 16;
+  const int blk = active ? tile >> 4 : 0, tr = (tile >> 2) & 3, tcI = tile & 3;
+  const int i = blk + D, j = blk;
+  float acc[16];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+  if (active) {
+    const int k0 = 16 * j + part * KN, r0 = 16 * i + 4 * tr, c0 = 16 * j + 4 * tcI;
+    float4 l4[KN], t4[KN];
+#pragma unroll
+    for (int m = 0; m < KN; ++m) {
+      l4[m] = *reinterpret_cast<const float4 *>(&LT[(k0 + m) * 64 + r0]);
+      t4[m] = *reinterpret_cast<const float4 *>(&Tf[(k0 + m) * 64 + c0]);
+    }
+#pragma unroll
+    for (int m = 0; m < KN; ++m) {
+      const float la[4] = {l4[m].x, l4[m].y, l4[m].z, l4[m].w};
+      const float ta[4] = {t4[m].x, t4[m].y, t4[m].z, t4[m].w};
+#pragma unroll
+      for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+        for (int b2 = 0; b2 < 4; ++b2) acc[4 * a2 + b2] = fmaf(la[a2], ta[b2], acc[4 * a2 + b2]);
+    }
+  }
+#pragma unroll
+  for (int off = 1; off < KS; off <<= 1)
+#pragma unroll
+    for (int t = 0; t < 16; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+  if (active && part == 0) {
+#pragma unroll
+    for (int a2 = 0; a2 < 4; ++a2)
+      *reinterpret_cast<float4 *>(&Xs[blk * 256 + (4 * tr + a2) * 16 + 4 * tcI]) =
+          make_float4(acc[4 * a2], acc[4 * a2 + 1], acc[4 * a2 + 2], acc[4 * a2 + 3]);
+  }
+  tc::named_bar(1, 128);
+#pragma unroll
+  for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+  if (active) {
+    const int m0 = part * KN2;
+    float4 l4[KN2], x4[KN2];
+#pragma unroll
+    for (int m = 0; m < KN2; ++m) {
+      l4[m] = *reinterpret_cast<const float4 *>(&TDT[i * 256 + (m0 + m) * 16 + 4 * tr]);
+      x4[m] = *reinterpret_cast<const float4 *>(&Xs[blk * 256 + (m0 + m) * 16 + 4 * tcI]);
+    }
+#pragma unroll
+    for (int m = 0; m < KN2; ++m) {
+      const float la[4] = {l4[m].x, l4[m].y, l4[m].z, l4[m].w};
+      const float xa[4] = {x4[m].x, x4[m].y, x4[m].z, x4[m].w};
+#pragma unroll
+      for (int a2 = 0; a2 < 4; ++a2)
+#pragma unroll
+        for (int b2 = 0; b2 < 4; ++b2) acc[4 * a2 + b2] = fmaf(la[a2], xa[b2], acc[4 * a2 + b2]);
+    }
+  }
+#pragma unroll
+  for (int off = 1; off < KS; off <<= 1)
+#pragma unroll
+    for (int t = 0; t < 16; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+  if (active && part == 0) {
+#pragma unroll
+    for (int a2 = 0; a2 < 4; ++a2)
+      *reinterpret_cast<float4 *>(&Tf[(16 * i + 4 * tr + a2) * 64 + 16 * j + 4 * tcI]) =
+          make_float4(-acc[4 * a2], -acc[4 * a2 + 1], -acc[4 * a2 + 2], -acc[4 * a2 + 3]);
+  }
+  tc::named_bar(1, 128);
 }
 
 // Every lane has finished its shared/tensor-memory work for this hand-off (and fenced it);
@@ -136,7 +215,8 @@ template <bool OUT_F32>
 __global__ void __launch_bounds__(NT, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, PrefillArgs a) {
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_o, PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -177,7 +257,17 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Hand-off waits.  Critical-path waits poll (mbarrier.test_wait); in the prep and state
+  // roles only one leader thread polls while the rest of the role blocks in a hardware
+  // named barrier, which costs no issue slots and releases as soon as the leader arrives.
   auto wait = [&](int i, uint32_t parity) { tc::mbar_wait(bar(i), parity, abort_flag); };
+  auto wait_sleep = [&](int i, uint32_t parity) {
+    tc::mbar_wait_sleep(bar(i), parity, abort_flag);
+  };
+  auto role_wait = [&](int i, uint32_t parity, bool leader, uint32_t bar_id, uint32_t nthreads) {
+    if (leader) tc::mbar_wait(bar(i), parity, abort_flag);
+    tc::named_bar(bar_id, nthreads);
+  };
 
   if (wg == 0) {
     // =========================================================== producer roles
@@ -188,14 +278,14 @@ __global__ void __launch_bounds__(NT, 1)
       for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1, z = zbase + bos + c * C;
         const uint32_t dst = sb + OFF_QK + (uint32_t)s * QK_BYTES;
-        if (c >= 2) wait(B_QK_EMPTY + s, (((uint32_t)c >> 1) & 1u) ^ 1u);
+        if (c >= 2) wait_sleep(B_QK_EMPTY + s, (((uint32_t)c >> 1) & 1u) ^ 1u);
         if (*abort_flag) break;
         tc::mbar_arrive_expect_tx(bar(B_QK_FULL + s), QK_BYTES);
         tc::tma_load_3d(dst + QK_K0, &tm_k, bar(B_QK_FULL + s), 0, hq, z);
         tc::tma_load_3d(dst + QK_K1, &tm_k, bar(B_QK_FULL + s), 64, hq, z);
         tc::tma_load_3d(dst + QK_Q0, &tm_q, bar(B_QK_FULL + s), 0, hq, z);
         tc::tma_load_3d(dst + QK_Q1, &tm_q, bar(B_QK_FULL + s), 64, hq, z);
-        if (c >= 1) wait(B_V_EMPTY, (uint32_t)(c - 1) & 1u);
+        if (c >= 1) wait_sleep(B_V_EMPTY, (uint32_t)(c - 1) & 1u);
         if (*abort_flag) break;
         tc::mbar_arrive_expect_tx(bar(B_V_FULL), V_BYTES);
         tc::tma_load_3d(sb + OFF_V, &tm_v, bar(B_V_FULL), 0, h, z);
@@ -292,7 +382,10 @@ __global__ void __launch_bounds__(NT, 1)
       // ------------------------------------------------------- gates
       for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1, t0 = bos + c * C, L = min(C, eos - t0);
-        if (c >= 2) wait(B_GATE_EMPTY + s, ((uint32_t)(c - 2) >> 1) & 1u);
+        if (c >= 2) {
+          if (lane == 0) wait_sleep(B_GATE_EMPTY + s, ((uint32_t)(c - 2) >> 1) & 1u);
+          __syncwarp();
+        }
         float g0 = 0.f, g1 = 0.f, b0 = 0.f, b1 = 0.f;
         const size_t i0 = ((size_t)zbase + t0 + lane) * a.Hv + h;
         if (lane < L) {
@@ -319,10 +412,10 @@ __global__ void __launch_bounds__(NT, 1)
         gs[lane + 32] = g1 * LOG2E;
         gs[64 + lane] = b0;
         gs[96 + lane] = b1;
-        gs[128 + lane] = exp2f(g0 * LOG2E);
-        gs[160 + lane] = exp2f(g1 * LOG2E);
-        gs[192 + lane] = exp2f((blast - g0) * LOG2E);
-        gs[224 + lane] = exp2f((blast - g1) * LOG2E);
+        gs[128 + lane] = tc::ex2(g0 * LOG2E);
+        gs[160 + lane] = tc::ex2(g1 * LOG2E);
+        gs[192 + lane] = tc::ex2((blast - g0) * LOG2E);
+        gs[224 + lane] = tc::ex2((blast - g1) * LOG2E);
         warp_arrive(bar(B_GATE_FULL + s), lane);
       }
     }
@@ -336,8 +429,8 @@ __global__ void __launch_bounds__(NT, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
       const float *gs = gates + 256 * s;
-      wait(B_GATE_FULL + s, ((uint32_t)c >> 1) & 1u);
-      wait(B_G_FULL, (uint32_t)c & 1u);
+      if (pt == 0) wait(B_GATE_FULL + s, ((uint32_t)c >> 1) & 1u);
+      role_wait(B_G_FULL, (uint32_t)c & 1u, pt == 0, 1, 128);
       tc::tc_fence_after();
       // ---- L^T (TMEM lanes 0-63 hold rows r of K K^T): L_rs = beta_r Gamma_rs (k_r . k_s), s < r ----
       if (q4 < 2) {
@@ -355,7 +448,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int cc = 0; cc < 32; ++cc) {
             const int s_ = 32 * half + cc;
-            LT[s_ * 64 + r] = (s_ < r) ? bt * exp2f(br - bs[cc]) * v[cc] : 0.f;
+            LT[s_ * 64 + r] = (s_ < r) ? bt * tc::ex2(br - bs[cc]) * v[cc] : 0.f;
           }
         }
       }
@@ -381,71 +474,11 @@ __global__ void __launch_bounds__(NT, 1)
       }
       tc::named_bar(1, 128);
       // ---- block merges by distance d = i - j:  X = sum_{k=j}^{i-1} L_ik T_kj,  T_ij = -T_ii X.
-      //      4x4 register tiles, the K range split over ks adjacent lanes (shuffle-reduced). ----
-#pragma unroll 1
-      for (int d = 1; d < 4; ++d) {
-        const int nb = 4 - d;                   // blocks in this round
-        const int ks = d == 1 ? 2 : (d == 2 ? 4 : 8);
-        const int item = pt, part = item & (ks - 1), tile = item / ks;
-        const bool active = tile < nb * 16;
-        const int blk = tile >> 4, tr = (tile >> 2) & 3, tcI = tile & 3;
-        const int i = blk + d, j = blk;
-        float acc[16];
-#pragma unroll
-        for (int t = 0; t < 16; ++t) acc[t] = 0.f;
-        if (active) {
-          const int kn = 16 * d / ks, k0 = 16 * j + part * kn;
-          const int r0 = 16 * i + 4 * tr, c0 = 16 * j + 4 * tcI;
-          for (int m = 0; m < kn; ++m) {
-            const float4 l4 = *reinterpret_cast<const float4 *>(&LT[(k0 + m) * 64 + r0]);
-            const float4 t4 = *reinterpret_cast<const float4 *>(&Tf[(k0 + m) * 64 + c0]);
-            const float la[4] = {l4.x, l4.y, l4.z, l4.w}, ta[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-            for (int a2 = 0; a2 < 4; ++a2)
-#pragma unroll
-              for (int b2 = 0; b2 < 4; ++b2) acc[4 * a2 + b2] += la[a2] * ta[b2];
-          }
-        }
-#pragma unroll
-        for (int off = 1; off < 8; off <<= 1)
-          if (off < ks)
-#pragma unroll
-            for (int t = 0; t < 16; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-        if (active && part == 0) {
-#pragma unroll
-          for (int a2 = 0; a2 < 4; ++a2)
-            *reinterpret_cast<float4 *>(&Xs[blk * 256 + (4 * tr + a2) * 16 + 4 * tcI]) =
-                make_float4(acc[4 * a2], acc[4 * a2 + 1], acc[4 * a2 + 2], acc[4 * a2 + 3]);
-        }
-        tc::named_bar(1, 128);
-#pragma unroll
-        for (int t = 0; t < 16; ++t) acc[t] = 0.f;
-        if (active) {  // T_ij = -T_ii X  (K = 16 split over ks lanes)
-          const int kn = 16 / ks, m0 = part * kn;
-#pragma unroll 1
-          for (int m = m0; m < m0 + kn; ++m) {
-            const float4 l4 = *reinterpret_cast<const float4 *>(&TDT[i * 256 + m * 16 + 4 * tr]);
-            const float4 x4 = *reinterpret_cast<const float4 *>(&Xs[blk * 256 + m * 16 + 4 * tcI]);
-            const float la[4] = {l4.x, l4.y, l4.z, l4.w}, xa[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll
-            for (int a2 = 0; a2 < 4; ++a2)
-#pragma unroll
-              for (int b2 = 0; b2 < 4; ++b2) acc[4 * a2 + b2] += la[a2] * xa[b2];
-          }
-        }
-#pragma unroll
-        for (int off = 1; off < 8; off <<= 1)
-          if (off < ks)
-#pragma unroll
-            for (int t = 0; t < 16; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-        if (active && part == 0) {
-#pragma unroll
-          for (int a2 = 0; a2 < 4; ++a2)
-            *reinterpret_cast<float4 *>(&Tf[(16 * i + 4 * tr + a2) * 64 + 16 * j + 4 * tcI]) =
-                make_float4(-acc[4 * a2], -acc[4 * a2 + 1], -acc[4 * a2 + 2], -acc[4 * a2 + 3]);
-        }
-        tc::named_bar(1, 128);
-      }
+      //      4x4 register tiles, the K range split over KS adjacent lanes (shuffle-reduced);
+      //      loops are fully unrolled so that every shared load is issued up front. ----
+      merge_round<1>(pt, LT, Tf, Xs, TDT);
+      merge_round<2>(pt, LT, Tf, Xs, TDT);
+      merge_round<3>(pt, LT, Tf, Xs, TDT);
       // ---- T diag(beta) (over L's region) and T diag(beta gamma) (over the scratch) ----
       for (int e = pt; e < 64 * 8; e += 128) {
         const int r = e >> 3, q = e & 7;
@@ -465,7 +498,7 @@ __global__ void __launch_bounds__(NT, 1)
       tc::fence_async_smem();
       warp_arrive(bar(B_TB_FULL), lane);
       // ---- P rows (TMEM lanes 64-127): scale Gamma_rs (q_r . k_s), s <= r ----
-      if (c > 0) wait(B_H_FULL, (uint32_t)(c - 1) & 1u);  // Ob(c-1) has read P
+      if (c > 0) role_wait(B_H_FULL, (uint32_t)(c - 1) & 1u, pt == 0, 1, 128);  // Ob(c-1) read P
       if (q4 >= 2) {
         const int r = row - 64;
         const float br = gs[r];
@@ -476,7 +509,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int cc = 0; cc < 32; ++cc) {
             const int s_ = 32 * half + cc;
-            v[cc] = (s_ <= r) ? a.scale * exp2f(br - gs[s_]) * v[cc] : 0.f;
+            v[cc] = (s_ <= r) ? a.scale * tc::ex2(br - gs[s_]) * v[cc] : 0.f;
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q)
@@ -488,7 +521,7 @@ __global__ void __launch_bounds__(NT, 1)
       warp_arrive(bar(B_P_FULL), lane);
       warp_arrive(bar(B_G_EMPTY), lane);
       // ---- -W^T (TMEM lane i, 64 values of r) -> MN-major B tile over T's region ----
-      wait(B_W_FULL, (uint32_t)c & 1u);
+      role_wait(B_W_FULL, (uint32_t)c & 1u, pt == 0, 1, 128);
       tc::tc_fence_after();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -525,8 +558,12 @@ __global__ void __launch_bounds__(NT, 1)
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1, t0 = bos + c * C, L = min(C, eos - t0);
       const float *gs = gates + 256 * s;
-      wait(B_GATE_FULL + s, ((uint32_t)c >> 1) & 1u);
-      wait(B_DMMA_FULL, (uint32_t)c & 1u);
+      const int st = tid - 256;
+      if (st == 0) {
+        tc::bulk_wait_read();  // the previous chunk's output store has left shared memory
+        wait(B_GATE_FULL + s, ((uint32_t)c >> 1) & 1u);
+      }
+      role_wait(B_DMMA_FULL, (uint32_t)c & 1u, st == 0, 2, 256);
       tc::tc_fence_after();
       // ---- Delta^T, Delta~^T -> bf16 hi/lo K-major A tiles (row j, columns r of this half) ----
 #pragma unroll
@@ -547,10 +584,16 @@ __global__ void __launch_bounds__(NT, 1)
       tc::tc_fence_before();
       warp_arrive(bar(B_D_FULL), lane);
       warp_arrive(bar(B_DU_EMPTY), lane);
-      wait(B_H_FULL, (uint32_t)c & 1u);
+      role_wait(B_H_FULL, (uint32_t)c & 1u, st == 0, 2, 256);
       tc::tc_fence_after();
-      // ---- outputs: O[r][j] = scale gamma_r Oa[j][r] + Ob[j][r] ----
+      // ---- outputs: O[r][j] = scale gamma_r Oa[j][r] + Ob[j][r].  A full chunk is staged in
+      //      shared memory (over the Delta^T tiles, free until the next Delta epilogue) and
+      //      written by one TMA store; a partial last chunk is stored row by row so that no
+      //      token past the end of the sequence is touched. ----
       {
+        using OutT = typename std::conditional<OUT_F32, float, __nv_bfloat16>::type;
+        OutT *stage_o = reinterpret_cast<OutT *>(smem + OFF_DH);  // [64][DV]
+        const bool full = (L == C);
         const size_t obase = ((size_t)zbase + t0) * a.Hv + h;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -561,14 +604,20 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
           for (int cc = 0; cc < 16; ++cc) {
             const int r = r0 + cc;
-            if (r < L) {
-              const float val = a.scale * gs[128 + r] * oa[cc] + ob[cc];
-              const size_t off = (obase + (size_t)r * a.Hv) * DV + row;
-              if constexpr (OUT_F32)
-                static_cast<float *>(a.o)[off] = val;
-              else
-                static_cast<__nv_bfloat16 *>(a.o)[off] = __float2bfloat16_rn(val);
+            const float val = a.scale * gs[128 + r] * oa[cc] + ob[cc];
+            if (full) {
+              io<OutT>::st(stage_o + r * DV + row, val);
+            } else if (r < L) {
+              io<OutT>::st(static_cast<OutT *>(a.o) + (obase + (size_t)r * a.Hv) * DV + row, val);
             }
+          }
+        }
+        if (full) {
+          tc::fence_async_smem();
+          tc::named_bar(2, 256);
+          if (st == 0) {
+            tc::tma_store_3d(&tm_o, sb + OFF_DH, 0, h, zbase + t0);
+            tc::bulk_commit();
           }
         }
       }
@@ -591,6 +640,7 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
       for (int m = 0; m < 64; ++m) a.state_out[st_off + (size_t)(64 * swg + m) * DV + row] = Hr[m];
     }
+    if (tid == 256) tc::bulk_wait_all();
   }
 
   tc::tc_fence_before();
@@ -635,6 +685,20 @@ inline bool make_map(CUtensorMap *m, const void *base, int d, int heads, long lo
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output o [rows = B*T][heads][d] (fp32 or bf16), box d x 1 x 64, no swizzle (row-major tile).
+inline bool make_map_out(CUtensorMap *m, void *base, int d, int heads, long long rows, bool f32) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int es_bytes = f32 ? 4 : 2;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * es_bytes, (cuuint64_t)heads * d * es_bytes};
+  const cuuint32_t box[3] = {(cuuint32_t)d, 1, 64};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base,
+             dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tck
 
 inline bool tc_supported(int dk, int dv) { return dk == 128 && dv == 128; }
@@ -646,16 +710,17 @@ inline cudaError_t tc_dispatch(int dk, int dv, bool out_f32, const PrefillArgs &
     return out_f32 ? launch_chunk_simt<128, 128, __nv_bfloat16, float>(a, N, stream)
                    : launch_chunk_simt<128, 128, __nv_bfloat16, __nv_bfloat16>(a, N, stream);
   }
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const long long rows = (long long)a.B * a.T;
   if (!tck::make_map(&mq, a.q, dk, a.Hqk, rows) || !tck::make_map(&mk, a.k, dk, a.Hqk, rows) ||
-      !tck::make_map(&mv, a.v, dv, a.Hv, rows))
+      !tck::make_map(&mv, a.v, dv, a.Hv, rows) ||
+      !tck::make_map_out(&mo, a.o, dv, a.Hv, rows, out_f32))
     return cudaErrorInvalidValue;
   auto kern = out_f32 ? tck::chunk_tc_kernel<true> : tck::chunk_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tck::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)N * (unsigned)a.Hv, tck::NT, tck::SMEM_BYTES, stream>>>(mq, mk, mv, a);
+  kern<<<(unsigned)N * (unsigned)a.Hv, tck::NT, tck::SMEM_BYTES, stream>>>(mq, mk, mv, mo, a);
   return cudaGetLastError();
 }
 
