@@ -127,79 +127,89 @@ __device__ __forceinline__ void st_row_chunk_split(uint32_t tile_hi, uint32_t ti
   st_row_chunk(tile_lo, row, chunk, lo);
 }
 
-// One round of the block merges of T = (I + L)^-1 (blocks of 16; distance D = i - j):
-//   X_i = sum_{k=j}^{i-1} L_ik T_kj,   T_ij = -T_ii X_i   for the 4 - D blocks (i, i - D).
-// 128 threads; a thread owns a 4x4 tile of one block and 1/KS of the K range.
-template <int D>
-__device__ __forceinline__ void merge_round(int pt, const float *LT, float *Tf, float *Xs,
-                                            const float *TDT) {
-  constexpr int NB = 4 - D, KS = D == 1 ? 2 : (D == 2 ? 4 : 8);
-  constexpr int KN = 16 * D / KS, KN2 = 16 / KS;
-  const int part = pt & (KS - 1), tile = pt / KS;
-  const bool active = tile < NB * 16;
-  const int blk = active ? tile >> 4 : 0, tr = (tile >> 2) & 3, tcI = tile & 3;
-  const int i = blk + D, j = blk;
-  float acc[16];
+// Block merges of T = (I + L)^-1 (64 x 64; blocks of 16), 128 threads, two rounds:
+//   A: T_10 = -T_11 (L_10 T_00), T_32 = -T_33 (L_32 T_22)        (16 -> 32, 2x2 tiles)
+//   B: T_BA = -T_BB (L_BA T_AA) for the 32x32 halves A, B        (32 -> 64, 2x4 tiles)
+// Register tiles with float2/float4 shared operands; no K splits, so no shuffles.
+// In: LT = L^T [64][64]; Tf [64][64] with the four 16x16 diagonal blocks of T; TDT [4][16][16] =
+// the diagonal blocks transposed.  Scratch: XA [2][16][16], XB [32][32], TBBT [32][32].
+// Out: Tf lower blocks complete.
+__device__ __forceinline__ void merges_2round(int pt, const float *LT, float *Tf, float *XA,
+                                              float *XB, const float *TDT, float *TBBT) {
+  // ---- round A: T_10 = -T_11 (L_10 T_00), T_32 = -T_33 (L_32 T_22); 2x2 tiles ----
+  {
+    const int b = pt >> 6, lt = pt & 63, tr = lt >> 3, tcl = lt & 7;  // b: 0 -> (1,0), 1 -> (3,2)
+    const int i = 2 * b + 1, j = 2 * b;
+    const int r0 = 16 * i + 2 * tr, c0 = 16 * j + 2 * tcl;
+    float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
 #pragma unroll
-  for (int t = 0; t < 16; ++t) acc[t] = 0.f;
-  if (active) {
-    const int k0 = 16 * j + part * KN, r0 = 16 * i + 4 * tr, c0 = 16 * j + 4 * tcI;
-    float4 l4[KN], t4[KN];
-#pragma unroll
-    for (int m = 0; m < KN; ++m) {
-      l4[m] = *reinterpret_cast<const float4 *>(&LT[(k0 + m) * 64 + r0]);
-      t4[m] = *reinterpret_cast<const float4 *>(&Tf[(k0 + m) * 64 + c0]);
+    for (int m = 0; m < 16; ++m) {
+      const float2 l = *reinterpret_cast<const float2 *>(&LT[(16 * j + m) * 64 + r0]);
+      const float2 t = *reinterpret_cast<const float2 *>(&Tf[(16 * j + m) * 64 + c0]);
+      a00 = fmaf(l.x, t.x, a00); a01 = fmaf(l.x, t.y, a01);
+      a10 = fmaf(l.y, t.x, a10); a11 = fmaf(l.y, t.y, a11);
     }
+    float *X = XA + b * 256;
+    *reinterpret_cast<float2 *>(&X[(2 * tr) * 16 + 2 * tcl]) = make_float2(a00, a01);
+    *reinterpret_cast<float2 *>(&X[(2 * tr + 1) * 16 + 2 * tcl]) = make_float2(a10, a11);
+    tc::named_bar(1, 128);
+    a00 = a01 = a10 = a11 = 0.f;
 #pragma unroll
-    for (int m = 0; m < KN; ++m) {
-      const float la[4] = {l4[m].x, l4[m].y, l4[m].z, l4[m].w};
-      const float ta[4] = {t4[m].x, t4[m].y, t4[m].z, t4[m].w};
-#pragma unroll
-      for (int a2 = 0; a2 < 4; ++a2)
-#pragma unroll
-        for (int b2 = 0; b2 < 4; ++b2) acc[4 * a2 + b2] = fmaf(la[a2], ta[b2], acc[4 * a2 + b2]);
+    for (int m = 0; m < 16; ++m) {  // T_ii^T[m][r] (zero for m > r)
+      const float2 l = *reinterpret_cast<const float2 *>(&TDT[i * 256 + m * 16 + 2 * tr]);
+      const float2 x = *reinterpret_cast<const float2 *>(&X[m * 16 + 2 * tcl]);
+      a00 = fmaf(l.x, x.x, a00); a01 = fmaf(l.x, x.y, a01);
+      a10 = fmaf(l.y, x.x, a10); a11 = fmaf(l.y, x.y, a11);
+    }
+    *reinterpret_cast<float2 *>(&Tf[(r0) * 64 + c0]) = make_float2(-a00, -a01);
+    *reinterpret_cast<float2 *>(&Tf[(r0 + 1) * 64 + c0]) = make_float2(-a10, -a11);
+    if (b == 1) {  // T_BB^T [m][r] (local indices): T_32^T block at m in 0..15, r in 16..31
+      TBBT[(2 * tcl) * 32 + 16 + 2 * tr] = -a00;     TBBT[(2 * tcl) * 32 + 17 + 2 * tr] = -a10;
+      TBBT[(2 * tcl + 1) * 32 + 16 + 2 * tr] = -a01; TBBT[(2 * tcl + 1) * 32 + 17 + 2 * tr] = -a11;
     }
   }
-#pragma unroll
-  for (int off = 1; off < KS; off <<= 1)
-#pragma unroll
-    for (int t = 0; t < 16; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-  if (active && part == 0) {
-#pragma unroll
-    for (int a2 = 0; a2 < 4; ++a2)
-      *reinterpret_cast<float4 *>(&Xs[blk * 256 + (4 * tr + a2) * 16 + 4 * tcI]) =
-          make_float4(acc[4 * a2], acc[4 * a2 + 1], acc[4 * a2 + 2], acc[4 * a2 + 3]);
+  {  // the rest of T_BB^T: diagonal blocks T_22^T, T_33^T and the zero block (m in 16..31, r in 0..15)
+    for (int e = pt; e < 768; e += 128) {
+      const int q = e >> 8, w = e & 255, m = w >> 4, r = w & 15;
+      if (q == 0) TBBT[m * 32 + r] = TDT[2 * 256 + m * 16 + r];
+      else if (q == 1) TBBT[(16 + m) * 32 + 16 + r] = TDT[3 * 256 + m * 16 + r];
+      else TBBT[(16 + m) * 32 + r] = 0.f;
+    }
   }
   tc::named_bar(1, 128);
+  // ---- round B: X = L_BA T_AA (rows 32..63, cols 0..31), 2x4 tiles; column block uniform per warp ----
+  {
+    const int cb = pt >> 6, lt = pt & 63, tr = lt >> 2, tcl = lt & 3;
+    const int r0 = 32 + 2 * tr, c0 = 16 * cb + 4 * tcl;
+    float acc[8];
 #pragma unroll
-  for (int t = 0; t < 16; ++t) acc[t] = 0.f;
-  if (active) {
-    const int m0 = part * KN2;
-    float4 l4[KN2], x4[KN2];
-#pragma unroll
-    for (int m = 0; m < KN2; ++m) {
-      l4[m] = *reinterpret_cast<const float4 *>(&TDT[i * 256 + (m0 + m) * 16 + 4 * tr]);
-      x4[m] = *reinterpret_cast<const float4 *>(&Xs[blk * 256 + (m0 + m) * 16 + 4 * tcI]);
+    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+    const int kbeg = 16 * cb;  // T_AA[k][c] = 0 for k < 16 when c >= 16
+#pragma unroll 4
+    for (int k = kbeg; k < 32; ++k) {
+      const float2 l = *reinterpret_cast<const float2 *>(&LT[k * 64 + r0]);
+      const float4 t = *reinterpret_cast<const float4 *>(&Tf[k * 64 + c0]);
+      acc[0] = fmaf(l.x, t.x, acc[0]); acc[1] = fmaf(l.x, t.y, acc[1]);
+      acc[2] = fmaf(l.x, t.z, acc[2]); acc[3] = fmaf(l.x, t.w, acc[3]);
+      acc[4] = fmaf(l.y, t.x, acc[4]); acc[5] = fmaf(l.y, t.y, acc[5]);
+      acc[6] = fmaf(l.y, t.z, acc[6]); acc[7] = fmaf(l.y, t.w, acc[7]);
     }
+    *reinterpret_cast<float4 *>(&XB[(2 * tr) * 32 + c0]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4 *>(&XB[(2 * tr + 1) * 32 + c0]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    tc::named_bar(1, 128);
 #pragma unroll
-    for (int m = 0; m < KN2; ++m) {
-      const float la[4] = {l4[m].x, l4[m].y, l4[m].z, l4[m].w};
-      const float xa[4] = {x4[m].x, x4[m].y, x4[m].z, x4[m].w};
-#pragma unroll
-      for (int a2 = 0; a2 < 4; ++a2)
-#pragma unroll
-        for (int b2 = 0; b2 < 4; ++b2) acc[4 * a2 + b2] = fmaf(la[a2], xa[b2], acc[4 * a2 + b2]);
+    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+#pragma unroll 4
+    for (int m = 0; m < 32; ++m) {  // T_BB^T[m][r] (zero for m > r)
+      const float2 l = *reinterpret_cast<const float2 *>(&TBBT[m * 32 + 2 * tr]);
+      const float4 x = *reinterpret_cast<const float4 *>(&XB[m * 32 + c0]);
+      acc[0] = fmaf(l.x, x.x, acc[0]); acc[1] = fmaf(l.x, x.y, acc[1]);
+      acc[2] = fmaf(l.x, x.z, acc[2]); acc[3] = fmaf(l.x, x.w, acc[3]);
+      acc[4] = fmaf(l.y, x.x, acc[4]); acc[5] = fmaf(l.y, x.y, acc[5]);
+      acc[6] = fmaf(l.y, x.z, acc[6]); acc[7] = fmaf(l.y, x.w, acc[7]);
     }
-  }
-#pragma unroll
-  for (int off = 1; off < KS; off <<= 1)
-#pragma unroll
-    for (int t = 0; t < 16; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
-  if (active && part == 0) {
-#pragma unroll
-    for (int a2 = 0; a2 < 4; ++a2)
-      *reinterpret_cast<float4 *>(&Tf[(16 * i + 4 * tr + a2) * 64 + 16 * j + 4 * tcI]) =
-          make_float4(-acc[4 * a2], -acc[4 * a2 + 1], -acc[4 * a2 + 2], -acc[4 * a2 + 3]);
+    *reinterpret_cast<float4 *>(&Tf[r0 * 64 + c0]) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+    *reinterpret_cast<float4 *>(&Tf[(r0 + 1) * 64 + c0]) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
   }
   tc::named_bar(1, 128);
 }
@@ -424,8 +434,8 @@ __global__ void __launch_bounds__(NT, 1)
     const int pt = tid - 128;  // 0..127
     float *LT = reinterpret_cast<float *>(smem + OFF_RL);  // L^T fp32 [64 s][64 r]
     float *Tf = reinterpret_cast<float *>(smem + OFF_RT);  // T fp32 [64][64], row-major
-    float *Xs = reinterpret_cast<float *>(smem + OFF_RX);  // merge scratch: 3 x [16][16]
-    float *TDT = Xs + 3 * 256;                             // diagonal blocks transposed [4][16 m][16 r]
+    float *Xs = reinterpret_cast<float *>(smem + OFF_RX);  // merge scratch [2][16][16] | TDT | XB | TBBT
+    float *TDT = Xs + 512;                                 // diagonal blocks transposed [4][16 m][16 r]
     for (int c = 0; c < nchunks; ++c) {
       const int s = c & 1;
       const float *gs = gates + 256 * s;
@@ -473,12 +483,8 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       tc::named_bar(1, 128);
-      // ---- block merges by distance d = i - j:  X = sum_{k=j}^{i-1} L_ik T_kj,  T_ij = -T_ii X.
-      //      4x4 register tiles, the K range split over KS adjacent lanes (shuffle-reduced);
-      //      loops are fully unrolled so that every shared load is issued up front. ----
-      merge_round<1>(pt, LT, Tf, Xs, TDT);
-      merge_round<2>(pt, LT, Tf, Xs, TDT);
-      merge_round<3>(pt, LT, Tf, Xs, TDT);
+      // ---- block merges (two rounds, see merges_2round) ----
+      merges_2round(pt, LT, Tf, Xs, Xs + 2048, TDT, Xs + 3072);
       // ---- T diag(beta) (over L's region) and T diag(beta gamma) (over the scratch) ----
       for (int e = pt; e < 64 * 8; e += 128) {
         const int r = e >> 3, q = e & 7;
@@ -568,11 +574,16 @@ __global__ void __launch_bounds__(NT, 1)
       // ---- Delta^T, Delta~^T -> bf16 hi/lo K-major A tiles (row j, columns r of this half) ----
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        float v[16], w[16];
+        float v[16], w[16], dt[16];  // dt: e^{b_C - b_r} for these 16 columns
         const int r0 = 32 * swg + 16 * part;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 d4 = reinterpret_cast<const float4 *>(gs + 192 + r0)[q];
+          dt[4 * q] = d4.x; dt[4 * q + 1] = d4.y; dt[4 * q + 2] = d4.z; dt[4 * q + 3] = d4.w;
+        }
         tc::tmem_ld16(tmem + lane_off + COL_DU + r0, v);
 #pragma unroll
-        for (int cc = 0; cc < 16; ++cc) w[cc] = v[cc] * gs[192 + r0 + cc];
+        for (int cc = 0; cc < 16; ++cc) w[cc] = v[cc] * dt[cc];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int ch = (r0 >> 3) + q;
@@ -597,14 +608,20 @@ __global__ void __launch_bounds__(NT, 1)
         const size_t obase = ((size_t)zbase + t0) * a.Hv + h;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          float oa[16], ob[16];
+          float oa[16], ob[16], gsc[16];  // gsc: scale * gamma_r for these 16 rows
           const int r0 = 32 * swg + 16 * part;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 g4 = reinterpret_cast<const float4 *>(gs + 128 + r0)[q];
+            gsc[4 * q] = a.scale * g4.x; gsc[4 * q + 1] = a.scale * g4.y;
+            gsc[4 * q + 2] = a.scale * g4.z; gsc[4 * q + 3] = a.scale * g4.w;
+          }
           tc::tmem_ld16(tmem + lane_off + COL_OA + r0, oa);
           tc::tmem_ld16(tmem + lane_off + COL_OB + r0, ob);
 #pragma unroll
           for (int cc = 0; cc < 16; ++cc) {
             const int r = r0 + cc;
-            const float val = a.scale * gs[128 + r] * oa[cc] + ob[cc];
+            const float val = gsc[cc] * oa[cc] + ob[cc];
             if (full) {
               io<OutT>::st(stage_o + r * DV + row, val);
             } else if (r < L) {
