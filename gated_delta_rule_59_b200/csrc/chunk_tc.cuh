@@ -106,7 +106,8 @@ enum Bar {
   B_D_FULL = 18,     // state (256) -> MMA
   B_DU_EMPTY = 19,   // state (256) -> MMA
   B_H_FULL = 20,     // MMA -> state, prep
-  NUM_BARS = 21
+  B_OA_EMPTY = 21,   // state (256) -> MMA: Oa/Ob accumulators have been read
+  NUM_BARS = 22
 };
 
 __device__ __forceinline__ void st_row_chunk(uint32_t tile, int row, int chunk, const float *v) {
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(NT, 1)
     // arrival counts: 1 = one thread (TMA expect_tx or tcgen05.commit), else one elected
     // lane per warp of the signalling group (gates 1, prep 4, state 8, prep + state 12)
     static constexpr uint16_t counts[NUM_BARS] = {1, 1, 1, 1, 1, 1, 1, 1, 12, 12, 1,
-                                                  4, 4, 4, 1, 4, 8, 1, 8, 8, 1};
+                                                  4, 4, 4, 1, 4, 8, 1, 8, 8, 1, 8};
     for (int i = 0; i < NUM_BARS; ++i) tc::mbar_init(bar(i), counts[i]);
     *abort_flag = 0;
     tc::fence_barrier_init();
@@ -303,37 +304,58 @@ __global__ void __launch_bounds__(NT, 1)
       }
     } else if (warp == 1 && lane == 0 && nchunks > 0) {
       // ------------------------------------------------------- MMA issuer
+      // Shared-memory descriptors are built once; per chunk only the stage base changes.
+      const uint64_t dKQ = tc::sdesc_sw128(sb + OFF_QK, 16, 1024);              // [K;Q], K (K-major)
+      const uint64_t dKmn = tc::sdesc_sw128(sb + OFF_QK + QK_K0, 16384, 1024);  // K (MN-major)
+      const uint64_t dQ = tc::sdesc_sw128(sb + OFF_QK + QK_Q0, 16, 1024);       // Q (K-major)
+      const uint64_t dV = tc::sdesc_sw128(sb + OFF_V, 8192, 1024);              // V (MN-major)
+      const uint64_t dTB = tc::sdesc_sw128(sb + OFF_RL, 16, 1024);              // T diag(beta) hi
+      const uint64_t dTBG = tc::sdesc_sw128(sb + OFF_RX, 16, 1024);             // T diag(beta gamma) hi
+      const uint64_t dW = tc::sdesc_sw128(sb + OFF_RT, 8192, 1024);             // -W^T (MN-major)
+      const uint64_t dDH = tc::sdesc_sw128(sb + OFF_DH, 16, 1024);
+      const uint64_t dDL = tc::sdesc_sw128(sb + OFF_DL, 16, 1024);
+      const uint64_t dDTH = tc::sdesc_sw128(sb + OFF_DTH, 16, 1024);
+      const uint64_t dDTL = tc::sdesc_sw128(sb + OFF_DTL, 16, 1024);
+      const uint64_t dPH = tc::sdesc_sw128(sb + OFF_P, 16, 1024);
+      const uint64_t dPL = tc::sdesc_sw128(sb + OFF_P + 8192, 16, 1024);
+      // descriptor address field is in 16-byte units
+      auto adv = [](uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); };
       auto issue_G = [&](int c) {
         const int s = c & 1;
         wait(B_QK_FULL + s, ((uint32_t)c >> 1) & 1u);
         if (c > 0) wait(B_G_EMPTY, (uint32_t)(c - 1) & 1u);
         if (*abort_flag) return;
         tc::tc_fence_after();
-        const uint32_t stg = sb + OFF_QK + (uint32_t)s * QK_BYTES;
+        const uint64_t d0 = adv(dKQ, (uint32_t)s * QK_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t d = tc::sdesc_sw128(stg + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024);
+          const uint64_t d = adv(d0, (kk >> 2) * 16384u + (kk & 3) * 32u);
           tc::mma_bf16(tmem + COL_G, d, d, ID_G, kk > 0);
         }
         tc::mma_commit(bar(B_G_FULL));
       };
       auto issue_WU = [&](int c) {
         wait(B_TB_FULL, (uint32_t)c & 1u);
+        if (*abort_flag) return;
+        tc::tc_fence_after();
+        const uint64_t dk = adv(dKmn, (uint32_t)(c & 1) * QK_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // W^T first: the prep role waits for it
+          const uint64_t ak = adv(dk, kk * 2048u);
+          tc::mma_bf16(tmem + COL_W, ak, adv(dTBG, kk * 32u), ID_MNK, kk > 0);
+          tc::mma_bf16(tmem + COL_W, ak, adv(dTBG, 8192u + kk * 32u), ID_MNK, 1);
+        }
+        tc::mma_commit(bar(B_W_FULL));
         wait(B_V_FULL, (uint32_t)c & 1u);
         if (c > 0) wait(B_DU_EMPTY, (uint32_t)(c - 1) & 1u);
         if (*abort_flag) return;
         tc::tc_fence_after();
-        const uint32_t stg = sb + OFF_QK + (uint32_t)(c & 1) * QK_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ak = tc::sdesc_sw128(stg + QK_K0 + kk * 2048u, 16384, 1024);
-          const uint64_t av = tc::sdesc_sw128(sb + OFF_V + kk * 2048u, 8192, 1024);
-          tc::mma_bf16(tmem + COL_W, ak, tc::sdesc_sw128(sb + OFF_RX + kk * 32u, 16, 1024), ID_MNK, kk > 0);
-          tc::mma_bf16(tmem + COL_W, ak, tc::sdesc_sw128(sb + OFF_RX + 8192 + kk * 32u, 16, 1024), ID_MNK, 1);
-          tc::mma_bf16(tmem + COL_DU, av, tc::sdesc_sw128(sb + OFF_RL + kk * 32u, 16, 1024), ID_MNK, kk > 0);
-          tc::mma_bf16(tmem + COL_DU, av, tc::sdesc_sw128(sb + OFF_RL + 8192 + kk * 32u, 16, 1024), ID_MNK, 1);
+          const uint64_t av = adv(dV, kk * 2048u);
+          tc::mma_bf16(tmem + COL_DU, av, adv(dTB, kk * 32u), ID_MNK, kk > 0);
+          tc::mma_bf16(tmem + COL_DU, av, adv(dTB, 8192u + kk * 32u), ID_MNK, 1);
         }
-        tc::mma_commit(bar(B_W_FULL));
         tc::mma_commit(bar(B_V_EMPTY));
       };
       auto issue_DO = [&](int c) {
@@ -341,38 +363,36 @@ __global__ void __launch_bounds__(NT, 1)
         wait(B_H0_FULL, (uint32_t)c & 1u);
         if (*abort_flag) return;
         tc::tc_fence_after();
-        const uint32_t stg = sb + OFF_QK + (uint32_t)(c & 1) * QK_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bw = tc::sdesc_sw128(sb + OFF_RT + kk * 2048u, 8192, 1024);
-          tc::mma_bf16_ta(tmem + COL_DU, tmem + COL_H0 + 8 * kk, bw, ID_KMN64, 1);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_bf16_ta(tmem + COL_DU, tmem + COL_H0 + 8 * kk, adv(dW, kk * 2048u), ID_KMN64, 1);
         tc::mma_commit(bar(B_DMMA_FULL));
+        if (c > 0) wait(B_OA_EMPTY, (uint32_t)(c - 1) & 1u);  // outputs of c-1 read out
+        tc::tc_fence_after();
+        const uint64_t dq = adv(dQ, (uint32_t)(c & 1) * QK_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bq =
-              tc::sdesc_sw128(stg + QK_Q0 + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024);
-          tc::mma_bf16_ta(tmem + COL_OA, tmem + COL_H0 + 8 * kk, bq, ID_KK64, kk > 0);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          tc::mma_bf16_ta(tmem + COL_OA, tmem + COL_H0 + 8 * kk,
+                          adv(dq, (kk >> 2) * 16384u + (kk & 3) * 32u), ID_KK64, kk > 0);
       };
       auto issue_HO = [&](int c) {
         wait(B_D_FULL, (uint32_t)c & 1u);
+        if (*abort_flag) return;
+        tc::tc_fence_after();
+        const uint64_t dk = adv(dKmn, (uint32_t)(c & 1) * QK_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // the state update first: it is on the critical path
+          const uint64_t bk = adv(dk, kk * 2048u);
+          tc::mma_bf16(tmem + COL_HU, adv(dDTH, kk * 32u), bk, ID_KMN128, kk > 0);
+          tc::mma_bf16(tmem + COL_HU, adv(dDTL, kk * 32u), bk, ID_KMN128, 1);
+        }
         wait(B_P_FULL, (uint32_t)c & 1u);
         if (*abort_flag) return;
         tc::tc_fence_after();
-        const uint32_t stg = sb + OFF_QK + (uint32_t)(c & 1) * QK_BYTES;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bk = tc::sdesc_sw128(stg + QK_K0 + kk * 2048u, 16384, 1024);
-          tc::mma_bf16(tmem + COL_HU, tc::sdesc_sw128(sb + OFF_DTH + kk * 32u, 16, 1024), bk, ID_KMN128, kk > 0);
-          tc::mma_bf16(tmem + COL_HU, tc::sdesc_sw128(sb + OFF_DTL + kk * 32u, 16, 1024), bk, ID_KMN128, 1);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t adh = tc::sdesc_sw128(sb + OFF_DH + kk * 32u, 16, 1024);
-          const uint64_t adl = tc::sdesc_sw128(sb + OFF_DL + kk * 32u, 16, 1024);
-          const uint64_t bph = tc::sdesc_sw128(sb + OFF_P + kk * 32u, 16, 1024);
-          const uint64_t bpl = tc::sdesc_sw128(sb + OFF_P + 8192 + kk * 32u, 16, 1024);
+          const uint64_t adh = adv(dDH, kk * 32u), adl = adv(dDL, kk * 32u);
+          const uint64_t bph = adv(dPH, kk * 32u), bpl = adv(dPL, kk * 32u);
           tc::mma_bf16(tmem + COL_OB, adh, bph, ID_KK64, kk > 0);
           tc::mma_bf16(tmem + COL_OB, adl, bph, ID_KK64, 1);
           tc::mma_bf16(tmem + COL_OB, adh, bpl, ID_KK64, 1);
@@ -597,6 +617,19 @@ __global__ void __launch_bounds__(NT, 1)
       warp_arrive(bar(B_DU_EMPTY), lane);
       role_wait(B_H_FULL, (uint32_t)c & 1u, st == 0, 2, 256);
       tc::tc_fence_after();
+      // ---- state: H = gamma_C H + Hupd; new H0^T operand ----
+      {
+        const float gC = gs[128 + 63];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float u[32];
+          tc::tmem_ld32(tmem + lane_off + COL_HU + 64 * swg + 32 * half, u);
+#pragma unroll
+          for (int m = 0; m < 32; ++m) Hr[32 * half + m] = gC * Hr[32 * half + m] + u[m];
+        }
+        store_h0();
+      }
+      warp_arrive(bar(B_H0_FULL), lane);  // the next chunk's Delta MMA may start
       // ---- outputs: O[r][j] = scale gamma_r Oa[j][r] + Ob[j][r].  A full chunk is staged in
       //      shared memory (over the Delta^T tiles, free until the next Delta epilogue) and
       //      written by one TMA store; a partial last chunk is stored row by row so that no
@@ -629,6 +662,8 @@ __global__ void __launch_bounds__(NT, 1)
             }
           }
         }
+        tc::tc_fence_before();
+        warp_arrive(bar(B_OA_EMPTY), lane);  // Oa / Ob read: the next Oa MMA may overwrite
         if (full) {
           tc::fence_async_smem();
           tc::named_bar(2, 256);
@@ -638,19 +673,6 @@ __global__ void __launch_bounds__(NT, 1)
           }
         }
       }
-      // ---- state: H = gamma_C H + Hupd; new H0^T operand ----
-      {
-        const float gC = gs[128 + 63];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float u[32];
-          tc::tmem_ld32(tmem + lane_off + COL_HU + 64 * swg + 32 * half, u);
-#pragma unroll
-          for (int m = 0; m < 32; ++m) Hr[32 * half + m] = gC * Hr[32 * half + m] + u[m];
-        }
-        store_h0();
-      }
-      warp_arrive(bar(B_H0_FULL), lane);
       warp_arrive(bar(B_GATE_EMPTY + s), lane);
     }
     if (a.state_out) {
