@@ -136,7 +136,8 @@ __device__ __forceinline__ void st_row_chunk_split(uint32_t tile_hi, uint32_t ti
 // the diagonal blocks transposed.  Scratch: XA [2][16][16], XB [32][32], TBBT [32][32].
 // Out: Tf lower blocks complete.
 __device__ __forceinline__ void merges_2round(int pt, const float *LT, float *Tf, float *XA,
-                                              float *XB, const float *TDT, float *TBBT) {
+                                              float *XB, const float *TDT, float *TBBT,
+                                              uint32_t nb = 1) {
   // ---- round A: T_10 = -T_11 (L_10 T_00), T_32 = -T_33 (L_32 T_22); 2x2 tiles ----
   {
     const int b = pt >> 6, lt = pt & 63, tr = lt >> 3, tcl = lt & 7;  // b: 0 -> (1,0), 1 -> (3,2)
@@ -153,7 +154,7 @@ __device__ __forceinline__ void merges_2round(int pt, const float *LT, float *Tf
     float *X = XA + b * 256;
     *reinterpret_cast<float2 *>(&X[(2 * tr) * 16 + 2 * tcl]) = make_float2(a00, a01);
     *reinterpret_cast<float2 *>(&X[(2 * tr + 1) * 16 + 2 * tcl]) = make_float2(a10, a11);
-    tc::named_bar(1, 128);
+    tc::named_bar(nb, 128);
     a00 = a01 = a10 = a11 = 0.f;
 #pragma unroll
     for (int m = 0; m < 16; ++m) {  // T_ii^T[m][r] (zero for m > r)
@@ -177,7 +178,7 @@ __device__ __forceinline__ void merges_2round(int pt, const float *LT, float *Tf
       else TBBT[(16 + m) * 32 + r] = 0.f;
     }
   }
-  tc::named_bar(1, 128);
+  tc::named_bar(nb, 128);
   // ---- round B: X = L_BA T_AA (rows 32..63, cols 0..31), 2x4 tiles; column block uniform per warp ----
   {
     const int cb = pt >> 6, lt = pt & 63, tr = lt >> 2, tcl = lt & 3;
@@ -197,7 +198,7 @@ __device__ __forceinline__ void merges_2round(int pt, const float *LT, float *Tf
     }
     *reinterpret_cast<float4 *>(&XB[(2 * tr) * 32 + c0]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
     *reinterpret_cast<float4 *>(&XB[(2 * tr + 1) * 32 + c0]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    tc::named_bar(1, 128);
+    tc::named_bar(nb, 128);
 #pragma unroll
     for (int t = 0; t < 8; ++t) acc[t] = 0.f;
 #pragma unroll 4
@@ -212,7 +213,7 @@ __device__ __forceinline__ void merges_2round(int pt, const float *LT, float *Tf
     *reinterpret_cast<float4 *>(&Tf[r0 * 64 + c0]) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
     *reinterpret_cast<float4 *>(&Tf[(r0 + 1) * 64 + c0]) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
   }
-  tc::named_bar(1, 128);
+  tc::named_bar(nb, 128);
 }
 
 // Every lane has finished its shared/tensor-memory work for this hand-off (and fenced it);
@@ -265,6 +266,7 @@ __global__ void __launch_bounds__(NT, 1)
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
+  __syncwarp();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
@@ -683,6 +685,7 @@ __global__ void __launch_bounds__(NT, 1)
   }
 
   tc::tc_fence_before();
+  __syncwarp();  // single-lane roles rejoin their warp before the CTA barrier
   __syncthreads();
   if (warp == 0) {
     tc::tc_fence_after();

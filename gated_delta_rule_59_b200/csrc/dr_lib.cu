@@ -12,6 +12,7 @@
 #include "decode.cuh"
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
+#include "chunk_pair.cuh"
 
 #define DR_VERSION_NUMBER 100  // 0.1.0
 
@@ -76,14 +77,14 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
       !aligned(beta, 4) || !aligned(cu_seqlens, 4))
     return DR_ERR_ALIGN;
   if (N == 0) return DR_OK;
-  if (N * Hv > 0x7fffffff) return DR_ERR_UNSUPPORTED;
+  if (N * Hv > 0x3fffffff) return DR_ERR_UNSUPPORTED;  // grid x of the CTA-pair launch: 2 N Hv
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   dr::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, (int)N, B, T, Hqk, Hv,
                     scale, o, state_out};
   cudaError_t e;
   if (in_dtype == DR_BF16 && dr::tc_supported(dk, dv)) {
-    e = dr::tc_dispatch(dk, dv, o_dtype == DR_F32, a, (int)N, s);
+    e = dr::prefill_tc_dispatch(dk, dv, o_dtype == DR_F32, a, (int)N, s);
   } else if (in_dtype == DR_F32) {
     e = simt_dispatch_out<float>(o_dtype, dk, dv, a, (int)N, s);
   } else {
