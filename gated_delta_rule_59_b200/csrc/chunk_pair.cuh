@@ -54,18 +54,20 @@ constexpr uint32_t WA_T = 16384;   // P hi | lo (shipped)
 constexpr uint32_t WA_X = 32768;   // T diag(beta gamma) hi | lo -> -W^T (shipped)
 constexpr uint32_t P_OFF_XS = P_OFF_WA + 2 * WA_BYTES;  // per instance: T rows 0-47 [48][64] fp32
 constexpr uint32_t XS_BYTES = 48 * 64 * 4;
+constexpr uint32_t P_OFF_DM = P_OFF_XS + 2 * XS_BYTES;  // per instance: diagonal-block inverses
+constexpr uint32_t DM_BYTES = 4 * 16 * 16 * 4;          //   [4][16 col][16 row], then T rows 48-63
+constexpr uint32_t P_OFF_GATES = P_OFF_DM + 2 * DM_BYTES;  // 2 slots x {bs2, beta, gam}[64]
 // state CTA
 constexpr uint32_t S_OFF_QK = 0;                      // two K/Q stages (outputs staged over them)
 constexpr uint32_t V_BYTES = 16384;
 constexpr uint32_t S_OFF_V = 2 * KQ_BYTES;            // two V stages
 constexpr uint32_t S_OFF_IN = S_OFF_V + 2 * V_BYTES;  // two incoming slots
 constexpr uint32_t IN_BYTES = 49152, IN_A_BYTES = 32768, IN_W = 32768, IN_W_BYTES = 16384;
-// both
-constexpr uint32_t OFF_GATES = 196608 + 2 * 12288;  // 2 slots x {bs2, beta, gam, dtil}[64]
-constexpr uint32_t OFF_BARS = OFF_GATES + 2 * 1024;
+constexpr uint32_t S_OFF_GATES = S_OFF_IN + 2 * IN_BYTES;  // 2 slots x {bs2, beta, gam, dtil}[64]
+// both: the barrier block sits at the same offset in the two CTAs (remote arrives address it)
+constexpr uint32_t OFF_BARS = P_OFF_GATES + 2 * 768;
 constexpr uint32_t SMEM_BYTES = OFF_BARS + 512 + 1024;  // + alignment slack
-static_assert(P_OFF_XS + 2 * XS_BYTES <= OFF_GATES, "prep shared memory");
-static_assert(S_OFF_IN + 2 * IN_BYTES <= OFF_GATES, "state shared memory");
+static_assert(S_OFF_GATES + 2 * 1024 <= OFF_BARS, "state shared memory");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ---- TMEM columns ----
@@ -83,7 +85,7 @@ enum Bar {
   P_GATE_EMPTY = 8,   // [2] instance (4 warps) -> gates warp
   P_G_FULL = 10,      // [2] issuer -> instance
   P_G_EMPTY = 12,     // [2] instance -> issuer
-  P_TBG_FULL = 14,    // [2] instance L warps (2) -> issuer (T diag(beta gamma) ready)
+  P_TBG_FULL = 14,    // [2] instance (4 warps) -> issuer (T diag(beta gamma) ready)
   P_W_FULL = 16,      // [2] issuer -> instance
   P_W_EMPTY = 18,     // [2] instance -> issuer
   P_IN_EMPTY = 20,    // [2] state CTA (remote) -> instance: the incoming slot is free
@@ -113,7 +115,7 @@ enum Bar {
 // bs2 = b log2(e), beta, gam = e^b, dtil = e^{b_C - b}.  Tokens past the end of the
 // sequence get g = beta = 0 (so they change nothing).  One warp.
 __device__ __forceinline__ void chunk_gates(const PrefillArgs &a, float *gs, int zbase, int t0,
-                                            int L, int h, int lane) {
+                                            int L, int h, int lane, bool with_dtil) {
   float g0 = 0.f, g1 = 0.f, b0 = 0.f, b1 = 0.f;
   const size_t i0 = ((size_t)zbase + t0 + lane) * a.Hv + h;
   if (lane < L) {
@@ -141,8 +143,10 @@ __device__ __forceinline__ void chunk_gates(const PrefillArgs &a, float *gs, int
   gs[96 + lane] = b1;
   gs[128 + lane] = tc::ex2(g0 * LOG2E);
   gs[160 + lane] = tc::ex2(g1 * LOG2E);
-  gs[192 + lane] = tc::ex2((blast - g0) * LOG2E);
-  gs[224 + lane] = tc::ex2((blast - g1) * LOG2E);
+  if (with_dtil) {
+    gs[192 + lane] = tc::ex2((blast - g0) * LOG2E);
+    gs[224 + lane] = tc::ex2((blast - g1) * LOG2E);
+  }
 }
 
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
@@ -158,11 +162,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o, PrefillArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Align by offsetting the shared array itself (not through an integer cast), so that every
+  // pointer derived from it stays in the shared address space: plain LDS/STS, not generic
+  // loads and stores.
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(smem);
-  float *gates = reinterpret_cast<float *>(smem + OFF_GATES);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BARS);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -187,8 +192,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
   if (tid == 0) {
     // arrival counts: 1 = one thread (TMA expect_tx, tcgen05.commit, copy expect_tx or a
     // remote arrive), else one elected lane per warp of the signalling group
-    static constexpr uint8_t pc[30] = {1, 1, 1, 1, 1, 1, 1, 1, 4, 4, 1, 1, 4, 4, 2,
-                                       2, 1, 1, 4, 4, 1, 1, 1, 1, 1, 1, 4, 4, 4, 4};
+    static constexpr uint8_t pc[30] = {1, 1, 1, 1, 1, 1, 1, 1, 4, 4, 1, 1, 4, 4, 4,
+                                       4, 1, 1, 4, 4, 1, 1, 1, 1, 1, 1, 4, 4, 4, 4};
     static constexpr uint8_t sc[22] = {1, 1, 1, 1, 1, 1, 1, 1, 1, 1, 12,
                                        12, 1, 1, 1, 1, 8, 1, 8, 1, 1, 4};
     if (rank == 0)
@@ -301,7 +306,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           if (lane == 0) wait_sleep(P_GATE_EMPTY + s, ((uint32_t)(c - 2) >> 1) & 1u);
           __syncwarp();
         }
-        chunk_gates(a, gates + 256 * s, zbase, t0, min(C, eos - t0), h, lane);
+        chunk_gates(a, reinterpret_cast<float *>(smem + P_OFF_GATES) + 192 * s, zbase, t0,
+                    min(C, eos - t0), h, lane, false);
         tck::warp_arrive(bar(P_GATE_FULL + s), lane);
       }
     } else if (warp == 3) {
@@ -332,7 +338,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       const uint32_t wa = sb + P_OFF_WA + (uint32_t)pi * WA_BYTES;
       float *LT = reinterpret_cast<float *>(smem + P_OFF_WA + pi * WA_BYTES + WA_LT);
       float *Xs = reinterpret_cast<float *>(smem + P_OFF_XS + pi * XS_BYTES);
-      const float *gs = gates + 256 * pi;
+      float *Dm = reinterpret_cast<float *>(smem + P_OFF_DM + pi * DM_BYTES);
+      const float *gs = reinterpret_cast<const float *>(smem + P_OFF_GATES) + 192 * pi;
       const uint32_t colG = 128u * (uint32_t)pi, colW = colG + 64;
       // G rows 0-63 are K K^T for instance 0 and Q K^T for instance 1: the warps on the
       // TMEM lanes of the K K^T rows build L and T, the other two build P.
@@ -371,38 +378,68 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           }
           if (rr == 0 && it > 0) wait_cl(P_INW_READ + pi, pph);  // X region: -W^T copy landed
           tc::named_bar(nbL, 64);
-          // ---- column rr of T = (I + L)^-1: forward substitution of (I + L) x = e_rr, in four
-          //      blocks of 16 rows.  The block being solved is in registers; finished rows go to
-          //      this thread's column of Xs (rows 0-47), so the loops stay compact. ----
+          // ---- T = (I + L)^-1 in 16-row blocks.  Phase A: the diagonal-block inverses
+          //      D_b = (I + L_bb)^-1, thread = (block b, column c), forward substitution ----
+          {
+            const int b = rr >> 4, cI = rr & 15, R = 16 * b;
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = (i == cI) ? 1.f : 0.f;
+#pragma unroll
+            for (int q = 0; q < 15; ++q) {
+              const float xq = x[q];
+#pragma unroll
+              for (int i = q + 1; i < 16; ++i) x[i] = fmaf(-LT[(R + q) * 64 + R + i], xq, x[i]);
+            }
+            float4 *dcol = reinterpret_cast<float4 *>(Dm + b * 256 + cI * 16);  // column-major
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              dcol[g] = make_float4(x[4 * g], x[4 * g + 1], x[4 * g + 2], x[4 * g + 3]);
+          }
+          tc::named_bar(nbL, 64);
+          // ---- Phase B: column j = rr, block by block: y = e_j - sum_{m < 16 b} L_{., m} x_m,
+          //      x_b = D_b y.  Rows 0-47 go to Xs ([row][column], the layout T is read in). ----
           float xb[16];
 #pragma unroll 1
           for (int b = 0; b < 4; ++b) {
+            float y[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) xb[i] = (16 * b + i == rr) ? 1.f : 0.f;
-#pragma unroll 2
-            for (int m = 0; m < 16 * b; ++m) {  // contributions of rows already solved
-              const float xm = Xs[m * 64 + rr];
-              const float4 *lm = reinterpret_cast<const float4 *>(LT + m * 64 + 16 * b);
+            for (int i = 0; i < 16; ++i) y[i] = (16 * b + i == rr) ? 1.f : 0.f;
+#pragma unroll 1
+            for (int m0 = 0; m0 < 16 * b; m0 += 4) {  // rows already solved, 4 at a time
+              float xm[4];
+              float4 l[4][4];
 #pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                const float4 l = lm[g];  // L_{r m} for r = 16 b + 4 g .. + 3
-                xb[4 * g + 0] = fmaf(-l.x, xm, xb[4 * g + 0]);
-                xb[4 * g + 1] = fmaf(-l.y, xm, xb[4 * g + 1]);
-                xb[4 * g + 2] = fmaf(-l.z, xm, xb[4 * g + 2]);
-                xb[4 * g + 3] = fmaf(-l.w, xm, xb[4 * g + 3]);
+              for (int u = 0; u < 4; ++u) {  // all loads of the group first
+                xm[u] = Xs[(m0 + u) * 64 + rr];
+                const float4 *lm = reinterpret_cast<const float4 *>(LT + (m0 + u) * 64 + 16 * b);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) l[u][g] = lm[g];  // L_{r m} for r = 16 b + 4 g .. + 3
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                  y[4 * g + 0] = fmaf(-l[u][g].x, xm[u], y[4 * g + 0]);
+                  y[4 * g + 1] = fmaf(-l[u][g].y, xm[u], y[4 * g + 1]);
+                  y[4 * g + 2] = fmaf(-l[u][g].z, xm[u], y[4 * g + 2]);
+                  y[4 * g + 3] = fmaf(-l[u][g].w, xm[u], y[4 * g + 3]);
+                }
               }
             }
+            // x_b = D_b y, column by column of D_b (16 independent accumulators)
 #pragma unroll
-            for (int q = 0; q < 15; ++q) {  // within the block
-              const float xq = xb[q];
-              const float4 *lq = reinterpret_cast<const float4 *>(LT + (16 * b + q) * 64 + 16 * b);
+            for (int i = 0; i < 16; ++i) xb[i] = 0.f;
 #pragma unroll
-              for (int g = (q + 1) >> 2; g < 4; ++g) {
-                const float4 l = lq[g];
-                if (4 * g + 0 > q) xb[4 * g + 0] = fmaf(-l.x, xq, xb[4 * g + 0]);
-                if (4 * g + 1 > q) xb[4 * g + 1] = fmaf(-l.y, xq, xb[4 * g + 1]);
-                if (4 * g + 2 > q) xb[4 * g + 2] = fmaf(-l.z, xq, xb[4 * g + 2]);
-                if (4 * g + 3 > q) xb[4 * g + 3] = fmaf(-l.w, xq, xb[4 * g + 3]);
+            for (int k = 0; k < 16; ++k) {
+              const float4 *dk = reinterpret_cast<const float4 *>(Dm + b * 256 + k * 16);
+#pragma unroll
+              for (int g = (k >> 2); g < 4; ++g) {  // D_b[i][k] = 0 for i < k
+                const float4 d = dk[g];
+                if (4 * g + 0 >= k) xb[4 * g + 0] = fmaf(d.x, y[k], xb[4 * g + 0]);
+                if (4 * g + 1 >= k) xb[4 * g + 1] = fmaf(d.y, y[k], xb[4 * g + 1]);
+                if (4 * g + 2 >= k) xb[4 * g + 2] = fmaf(d.z, y[k], xb[4 * g + 2]);
+                if (4 * g + 3 >= k) xb[4 * g + 3] = fmaf(d.w, y[k], xb[4 * g + 3]);
               }
             }
             if (b < 3) {
@@ -410,30 +447,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
               for (int i = 0; i < 16; ++i) Xs[(16 * b + i) * 64 + rr] = xb[i];
             }
           }
-          tc::named_bar(nbL, 64);  // all of L^T has been read: T diag(beta) goes over it
-          // ---- element (r, j = rr) of T diag(beta) -> L^T's region and of T diag(beta gamma)
-          //      -> X region, as bf16 hi/lo pairs in the K-major swizzled operand tiles ----
-          {
-            const float bj = gs[64 + rr], gj = gs[128 + rr];
-            const uint32_t cb = (uint32_t)(rr & 7) * 2u, ch = (uint32_t)(rr >> 3);
-            auto put = [&](int r, float xr) {
-              const uint32_t off = (uint32_t)r * 128u + ((ch ^ (uint32_t)(r & 7)) << 4) + cb;
-              const float tb = xr * bj, tbg = tb * gj;
-              const __nv_bfloat16 h1 = __float2bfloat16_rn(tb), h2 = __float2bfloat16_rn(tbg);
-              const __nv_bfloat16 l1 = __float2bfloat16_rn(tb - __bfloat162float(h1));
-              const __nv_bfloat16 l2 = __float2bfloat16_rn(tbg - __bfloat162float(h2));
-              tc::st_shared_u16(wa + WA_LT + off, __bfloat16_as_ushort(h1));
-              tc::st_shared_u16(wa + WA_LT + 8192 + off, __bfloat16_as_ushort(l1));
-              tc::st_shared_u16(wa + WA_X + off, __bfloat16_as_ushort(h2));
-              tc::st_shared_u16(wa + WA_X + 8192 + off, __bfloat16_as_ushort(l2));
-            };
-#pragma unroll 2
-            for (int r = 0; r < 48; ++r) put(r, Xs[r * 64 + rr]);
+          tc::named_bar(nbL, 64);  // every D_b has been used: T rows 48-63 go over them
 #pragma unroll
-            for (int i = 0; i < 16; ++i) put(48 + i, xb[i]);
-          }
-          tc::fence_async_smem();
-          tck::warp_arrive(bar(P_TBG_FULL + pi), lane);
+          for (int i = 0; i < 16; ++i) Dm[i * 64 + rr] = xb[i];
         } else {
           // ---- P rows: scale Gamma_rs (q_r . k_s), s <= r -> bf16 hi/lo tiles ----
           uint32_t u0[32], u1[32];
@@ -457,10 +473,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
             }
             tck::st_row_chunk_split(wa + WA_T, wa + WA_T + 8192, rr, q, v);
           }
-          tc::fence_async_smem();
         }
         tc::tc_fence_before();
-        tck::warp_arrive(bar(P_G_EMPTY + pi), lane);
+        tck::warp_arrive(bar(P_G_EMPTY + pi), lane);  // G has been read
+        tc::named_bar(nb, 128);  // T complete (rows 0-47 in Xs, 48-63 in Dm); L^T dead
+        // ---- T diag(beta) -> L^T's region, T diag(beta gamma) -> X region: 16-byte chunks
+        //      of 8 columns, bf16 hi/lo, by all four warps ----
+#pragma unroll 1
+        for (int e = pt; e < 64 * 8; e += 128) {
+          const int r = e >> 3, q = e & 7;
+          const float *trow = (r < 48) ? Xs + r * 64 : Dm + (r - 48) * 64;
+          const float4 ta = *reinterpret_cast<const float4 *>(trow + 8 * q);
+          const float4 tb4 = *reinterpret_cast<const float4 *>(trow + 8 * q + 4);
+          const float4 ba = reinterpret_cast<const float4 *>(gs + 64)[2 * q];
+          const float4 bb = reinterpret_cast<const float4 *>(gs + 64)[2 * q + 1];
+          const float4 ga = reinterpret_cast<const float4 *>(gs + 128)[2 * q];
+          const float4 gb = reinterpret_cast<const float4 *>(gs + 128)[2 * q + 1];
+          const float tv[8] = {ta.x, ta.y, ta.z, ta.w, tb4.x, tb4.y, tb4.z, tb4.w};
+          const float bv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+          const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+          float tb[8], tbg[8];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            tb[m] = (8 * q + m <= r) ? tv[m] * bv[m] : 0.f;
+            tbg[m] = tb[m] * gv[m];
+          }
+          tck::st_row_chunk_split(wa + WA_LT, wa + WA_LT + 8192, r, q, tb);
+          tck::st_row_chunk_split(wa + WA_X, wa + WA_X + 8192, r, q, tbg);
+        }
+        tc::fence_async_smem();
+        tck::warp_arrive(bar(P_TBG_FULL + pi), lane);
         tck::warp_arrive(bar(P_SHIP_A + pi), lane);
         // ---- -W^T (TMEM lane = key row k, 64 values of r) -> MN-major B tile over X ----
         role_wait(P_W_FULL + pi, ph, pt == 0, nb, 128);
@@ -612,7 +654,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           if (lane == 0) wait_sleep(S_GATE_EMPTY + s, ((uint32_t)(c - 2) >> 1) & 1u);
           __syncwarp();
         }
-        chunk_gates(a, gates + 256 * s, zbase, t0, min(C, eos - t0), h, lane);
+        chunk_gates(a, reinterpret_cast<float *>(smem + S_OFF_GATES) + 256 * s, zbase, t0,
+                    min(C, eos - t0), h, lane, true);
         tck::warp_arrive(bar(S_GATE_FULL + s), lane);
       }
     } else if (warp == 3) {
@@ -650,7 +693,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       }
       for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1;
-        const float *gs = gates + 256 * s;
+        const float *gs = reinterpret_cast<const float *>(smem + S_OFF_GATES) + 256 * s;
         if (st == 0) wait(S_GATE_FULL + s, ((uint32_t)c >> 1) & 1u);
         role_wait(S_DMMA_FULL, (uint32_t)c & 1u, st == 0, 3, 256);
         tc::tc_fence_after();
@@ -711,7 +754,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       const int ot = tid - 384;
       for (int c = 0; c < nchunks; ++c) {
         const int s = c & 1, t0 = bos + c * C, L = min(C, eos - t0);
-        const float *gs = gates + 256 * s;
+        const float *gs = reinterpret_cast<const float *>(smem + S_OFF_GATES) + 256 * s;
         if (ot == 0) wait(S_GATE_FULL + s, ((uint32_t)c >> 1) & 1u);
         role_wait(S_OB_FULL, (uint32_t)c & 1u, ot == 0, 4, 128);
         tc::tc_fence_after();

@@ -229,9 +229,11 @@ __global__ void __launch_bounds__(NT, 1)
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_o, PrefillArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // Align by offsetting the shared array itself (not through an integer cast), so that every
+  // pointer derived from it stays in the shared address space: plain LDS/STS, not generic
+  // loads and stores.
+  uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = tc::smem_u32(smem);
   float *gates = reinterpret_cast<float *>(smem + OFF_GATES);  // slot s: gates + 256 s
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BARS);
