@@ -51,12 +51,10 @@ constexpr uint32_t P_OFF_WA = P_NKQ * KQ_BYTES; // two instance work areas
 constexpr uint32_t WA_BYTES = 49152;
 constexpr uint32_t WA_LT = 0;      // L^T fp32 [64][64]       -> T diag(beta) hi | lo (shipped)
 constexpr uint32_t WA_T = 16384;   // P hi | lo (shipped)
-constexpr uint32_t WA_X = 32768;   // T diag(beta gamma) hi | lo -> -W^T (shipped)
-constexpr uint32_t P_OFF_XS = P_OFF_WA + 2 * WA_BYTES;  // per instance: T rows 0-47 [48][64] fp32
-constexpr uint32_t XS_BYTES = 48 * 64 * 4;
-constexpr uint32_t P_OFF_DM = P_OFF_XS + 2 * XS_BYTES;  // per instance: diagonal-block inverses
-constexpr uint32_t DM_BYTES = 4 * 16 * 16 * 4;          //   [4][16 col][16 row], then T rows 48-63
-constexpr uint32_t P_OFF_GATES = P_OFF_DM + 2 * DM_BYTES;  // 2 slots x {bs2, beta, gam}[64]
+constexpr uint32_t WA_X = 32768;   // merge scratch -> T diag(beta gamma) hi | lo -> -W^T (shipped)
+constexpr uint32_t P_OFF_TF = P_OFF_WA + 2 * WA_BYTES;  // per instance: T fp32 [64][64]
+constexpr uint32_t TF_BYTES = 64 * 64 * 4;
+constexpr uint32_t P_OFF_GATES = P_OFF_TF + 2 * TF_BYTES;  // 2 slots x {bs2, beta, gam}[64]
 // state CTA
 constexpr uint32_t S_OFF_QK = 0;                      // two K/Q stages (outputs staged over them)
 constexpr uint32_t V_BYTES = 16384;
@@ -337,8 +335,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       const uint32_t nbL = 3 + (uint32_t)pi;       // named barrier of its two L warps (64)
       const uint32_t wa = sb + P_OFF_WA + (uint32_t)pi * WA_BYTES;
       float *LT = reinterpret_cast<float *>(smem + P_OFF_WA + pi * WA_BYTES + WA_LT);
-      float *Xs = reinterpret_cast<float *>(smem + P_OFF_XS + pi * XS_BYTES);
-      float *Dm = reinterpret_cast<float *>(smem + P_OFF_DM + pi * DM_BYTES);
+      float *Tf = reinterpret_cast<float *>(smem + P_OFF_TF + pi * TF_BYTES);  // T, row-major
+      float *Xs = reinterpret_cast<float *>(smem + P_OFF_WA + pi * WA_BYTES + WA_X);  // scratch
+      float *TDT = Xs + 512;  // diagonal blocks of T transposed [4][16 m][16 r]
       const float *gs = reinterpret_cast<const float *>(smem + P_OFF_GATES) + 192 * pi;
       const uint32_t colG = 128u * (uint32_t)pi, colW = colG + 64;
       // G rows 0-63 are K K^T for instance 0 and Q K^T for instance 1: the warps on the
@@ -377,9 +376,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
             }
           }
           if (rr == 0 && it > 0) wait_cl(P_INW_READ + pi, pph);  // X region: -W^T copy landed
-          tc::named_bar(nbL, 64);
-          // ---- T = (I + L)^-1 in 16-row blocks.  Phase A: the diagonal-block inverses
-          //      D_b = (I + L_bb)^-1, thread = (block b, column c), forward substitution ----
+          tc::named_bar(nbL, 64);  // L^T complete
+          // ---- T = (I + L)^-1: the 16x16 diagonal blocks by forward substitution, one
+          //      column per thread (written to T and, transposed, to TDT) ----
           {
             const int b = rr >> 4, cI = rr & 15, R = 16 * b;
             float x[16];
@@ -391,65 +390,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
 #pragma unroll
               for (int i = q + 1; i < 16; ++i) x[i] = fmaf(-LT[(R + q) * 64 + R + i], xq, x[i]);
             }
-            float4 *dcol = reinterpret_cast<float4 *>(Dm + b * 256 + cI * 16);  // column-major
+#pragma unroll
+            for (int i = 0; i < 16; ++i) Tf[(R + i) * 64 + R + cI] = x[i];
+            float4 *trow = reinterpret_cast<float4 *>(TDT + b * 256 + cI * 16);
 #pragma unroll
             for (int g = 0; g < 4; ++g)
-              dcol[g] = make_float4(x[4 * g], x[4 * g + 1], x[4 * g + 2], x[4 * g + 3]);
+              trow[g] = make_float4(x[4 * g], x[4 * g + 1], x[4 * g + 2], x[4 * g + 3]);
           }
-          tc::named_bar(nbL, 64);
-          // ---- Phase B: column j = rr, block by block: y = e_j - sum_{m < 16 b} L_{., m} x_m,
-          //      x_b = D_b y.  Rows 0-47 go to Xs ([row][column], the layout T is read in). ----
-          float xb[16];
-#pragma unroll 1
-          for (int b = 0; b < 4; ++b) {
-            float y[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) y[i] = (16 * b + i == rr) ? 1.f : 0.f;
-#pragma unroll 1
-            for (int m0 = 0; m0 < 16 * b; m0 += 4) {  // rows already solved, 4 at a time
-              float xm[4];
-              float4 l[4][4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {  // all loads of the group first
-                xm[u] = Xs[(m0 + u) * 64 + rr];
-                const float4 *lm = reinterpret_cast<const float4 *>(LT + (m0 + u) * 64 + 16 * b);
-#pragma unroll
-                for (int g = 0; g < 4; ++g) l[u][g] = lm[g];  // L_{r m} for r = 16 b + 4 g .. + 3
-              }
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                  y[4 * g + 0] = fmaf(-l[u][g].x, xm[u], y[4 * g + 0]);
-                  y[4 * g + 1] = fmaf(-l[u][g].y, xm[u], y[4 * g + 1]);
-                  y[4 * g + 2] = fmaf(-l[u][g].z, xm[u], y[4 * g + 2]);
-                  y[4 * g + 3] = fmaf(-l[u][g].w, xm[u], y[4 * g + 3]);
-                }
-              }
-            }
-            // x_b = D_b y, column by column of D_b (16 independent accumulators)
-#pragma unroll
-            for (int i = 0; i < 16; ++i) xb[i] = 0.f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const float4 *dk = reinterpret_cast<const float4 *>(Dm + b * 256 + k * 16);
-#pragma unroll
-              for (int g = (k >> 2); g < 4; ++g) {  // D_b[i][k] = 0 for i < k
-                const float4 d = dk[g];
-                if (4 * g + 0 >= k) xb[4 * g + 0] = fmaf(d.x, y[k], xb[4 * g + 0]);
-                if (4 * g + 1 >= k) xb[4 * g + 1] = fmaf(d.y, y[k], xb[4 * g + 1]);
-                if (4 * g + 2 >= k) xb[4 * g + 2] = fmaf(d.z, y[k], xb[4 * g + 2]);
-                if (4 * g + 3 >= k) xb[4 * g + 3] = fmaf(d.w, y[k], xb[4 * g + 3]);
-              }
-            }
-            if (b < 3) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) Xs[(16 * b + i) * 64 + rr] = xb[i];
-            }
-          }
-          tc::named_bar(nbL, 64);  // every D_b has been used: T rows 48-63 go over them
-#pragma unroll
-          for (int i = 0; i < 16; ++i) Dm[i * 64 + rr] = xb[i];
         } else {
           // ---- P rows: scale Gamma_rs (q_r . k_s), s <= r -> bf16 hi/lo tiles ----
           uint32_t u0[32], u1[32];
@@ -476,13 +423,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         }
         tc::tc_fence_before();
         tck::warp_arrive(bar(P_G_EMPTY + pi), lane);  // G has been read
-        tc::named_bar(nb, 128);  // T complete (rows 0-47 in Xs, 48-63 in Dm); L^T dead
+        tc::named_bar(nb, 128);  // L^T and the diagonal blocks of T are complete
+        // ---- the off-diagonal blocks of T: two rounds of block merges (all four warps) ----
+        tck::merges_2round(pt, LT, Tf, Xs, Xs + 2048, TDT, Xs + 3072, nb);
         // ---- T diag(beta) -> L^T's region, T diag(beta gamma) -> X region: 16-byte chunks
         //      of 8 columns, bf16 hi/lo, by all four warps ----
 #pragma unroll 1
         for (int e = pt; e < 64 * 8; e += 128) {
           const int r = e >> 3, q = e & 7;
-          const float *trow = (r < 48) ? Xs + r * 64 : Dm + (r - 48) * 64;
+          const float *trow = Tf + r * 64;
           const float4 ta = *reinterpret_cast<const float4 *>(trow + 8 * q);
           const float4 tb4 = *reinterpret_cast<const float4 *>(trow + 8 * q + 4);
           const float4 ba = reinterpret_cast<const float4 *>(gs + 64)[2 * q];
