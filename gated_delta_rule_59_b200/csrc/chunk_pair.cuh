@@ -216,9 +216,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
   auto wait_sleep = [&](int i, uint32_t parity) {
     tc::mbar_wait_sleep(bar(i), parity, abort_flag);
   };
-  auto wait_cl = [&](int i, uint32_t parity) {
-    tc::mbar_wait_cluster(bar(i), parity, abort_flag);
-  };
+  // Phases completed from the partner CTA are polled at CTA scope too: incoming operands are
+  // made visible by the copies' complete_tx (as for any bulk or TMA copy), and the partner's
+  // acknowledgements publish no data.  (Cluster-scope acquire polls measured slower.)
+  auto wait_cl = [&](int i, uint32_t parity) { tc::mbar_wait(bar(i), parity, abort_flag); };
   // Loops of several threads never leave on the abort flag (threads could read it at
   // different times and part at a named barrier); after an abort every wait returns at once.
   auto role_wait = [&](int i, uint32_t parity, bool leader, uint32_t bar_id, uint32_t nthreads) {
