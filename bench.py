@@ -115,9 +115,20 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+# Sources each profiled kernel is compiled from (the first names the kernel in profiles/).
+KERNEL_SOURCES = {
+    "chunk_pair.cuh": ("chunk_pair.cuh", "chunk_tc.cuh", "tc_ptx.cuh"),
+    "decode.cuh": ("decode.cuh",),
+    "chunk_simt.cuh": ("chunk_simt.cuh",),
+}
+
+
 def kernel_source_sha(name: str) -> str:
-    with open(os.path.join(ROOT, "gated_delta_rule_59_b200", "csrc", name), "rb") as fh:
-        return hashlib.sha256(fh.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(name, (name,)):
+        with open(os.path.join(ROOT, "gated_delta_rule_59_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def profiled_traffic(kernel_file: str, workload: str):
@@ -254,7 +265,7 @@ def run_ours(args, dist: Dist):
     algo_bytes = prefill_bytes(B, T, Hqk, Hv, dk, dv, 2, 4, B, True)
     flops = prefill_flops(tokens * Hv, dk, dv)
     achieved = algo_bytes / (ms / 1e3) / 1e9
-    kfile = "chunk_tc.cuh" if kernel == "tc_bf16" else "chunk_simt.cuh"
+    kfile = "chunk_pair.cuh" if kernel == "tc_bf16" else "chunk_simt.cuh"
     roofline = {
         "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
         "frac": round(achieved / hbm_peak, 4),
