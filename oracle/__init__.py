@@ -7,7 +7,8 @@ nothing here imports the product path.
 
 Contents
   run(...)         token-by-token fp64 recurrence (C library ``liboracle.so``),
-                   three independent update forms (see ``dr_oracle.c``).
+                   three independent update forms (see ``dr_oracle.c``); optional
+                   q/k L2 normalisation first (``l2_normalize_rows``).
   chunk_ref        numpy fp64 chunk (UT/WY) form, used to pin the chunk algebra.
   brute            exact rational brute force on tiny inputs.
 
@@ -80,16 +81,32 @@ def _ptr(a, typ=ctypes.c_double):
     return a.ctypes.data_as(ctypes.POINTER(typ))
 
 
+def l2_normalize_rows(x):
+    """Each row (last axis) divided by its Euclidean norm, in fp64; an all-zero row stays zero.
+
+    "DeltaNet Attention" (class docstring) and "DeltaNet" (section "The Delta Rule") state that
+    queries and keys are L2-normalised before the rule; the "linear_attention" page draws it as
+    the ``qk_l2norm`` block in front of ``delta_rule``.  No epsilon is given: the plain quotient
+    is taken, with the zero row mapped to zero.
+    """
+    x = _f64(x)
+    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    return np.where(n > 0.0, x / np.where(n > 0.0, n, 1.0), 0.0)
+
+
 def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
-        form: int = 2, threads: int = 0):
+        form: int = 2, threads: int = 0, qk_l2norm: bool = False):
     """Token-by-token fp64 recurrence.
 
     q, k: [B, T, Hqk, dk]; v: [B, T, Hv, dv]; g, beta: [B, T, Hv] (g may be None);
     state_in: [N, Hv, dk, dv] or None (zeros); cu_seqlens: int [N+1] or None.
+    ``qk_l2norm``: q and k rows are L2-normalised first (``l2_normalize_rows``).
     Returns (o [B, T, Hv, dv], state_out [N, Hv, dk, dv]) as float64 numpy arrays.
     """
     lib = _load()
     q, k, v, g, beta, state_in = (_f64(a) for a in (q, k, v, g, beta, state_in))
+    if qk_l2norm:
+        q, k = np.ascontiguousarray(l2_normalize_rows(q)), np.ascontiguousarray(l2_normalize_rows(k))
     B, T, Hqk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     assert k.shape == q.shape and v.shape[:2] == (B, T) and beta.shape == (B, T, Hv)
@@ -117,7 +134,8 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
     return o, st
 
 
-def step(q, k, v, g, beta, state, scale: float = 1.0, form: int = 2, threads: int = 0):
+def step(q, k, v, g, beta, state, scale: float = 1.0, form: int = 2, threads: int = 0,
+         qk_l2norm: bool = False):
     """One decode step (T = 1) for every (batch, v-head).
 
     q, k: [B, Hqk, dk]; v: [B, Hv, dv]; g, beta: [B, Hv]; state: [B, Hv, dk, dv].
@@ -126,5 +144,5 @@ def step(q, k, v, g, beta, state, scale: float = 1.0, form: int = 2, threads: in
     q, k, v, beta, state = (_f64(a) for a in (q, k, v, beta, state))
     g = _f64(g)
     o, st = run(q[:, None], k[:, None], v[:, None], None if g is None else g[:, None],
-                beta[:, None], state, None, scale, form, threads)
+                beta[:, None], state, None, scale, form, threads, qk_l2norm)
     return o[:, 0], st

@@ -54,6 +54,14 @@ def test_head_dims(cuda_device, dk, dv, dtype):
     check_full(p, cuda_device, scale=dk ** -0.5)
 
 
+def test_many_units_several_cluster_waves(cuda_device):
+    """B=3, Hv=32: 96 (sequence, head) units = 192 CTAs of 2-CTA clusters, more than one wave
+    on 148 SMs; every output and final state against the oracle."""
+    p = inputs.prefill(3, 150, 16, 32, 128, 128, torch.bfloat16, gated=True, state_std=0.02,
+                       seed=77)
+    check_full(p, cuda_device)
+
+
 @pytest.mark.parametrize("group", [1, 2, 4])
 def test_gqa_groups(cuda_device, group):
     p = inputs.prefill(1, 130, 2, 2 * group, 128, 128, torch.bfloat16, gated=True,
