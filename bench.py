@@ -305,6 +305,27 @@ def run_ours(args, dist: Dist):
 
     secondary = {}
     if not args.no_secondary:
+        # the headline workload with the kernel's q/k L2 normalisation (DR_QK_L2NORM)
+        def l2_step(_):
+            dr.chunk_fwd(p.q, p.k, p.v, p.g, p.beta, p.state_in, None, o=o, state_out=st,
+                         qk_l2norm=True)
+
+        for i in range(2):
+            flush.zero_()
+            l2_step(i)
+        torch.cuda.synchronize()
+        assert dr.device_status(dev) == 0
+        dist.barrier()
+        l_durs = time_steps(l2_step, max(3, min(args.steps, 10)), stream, flush)
+        dist.barrier()
+        l_ms = dist.max(sum(l_durs) / len(l_durs), dev)
+        secondary["prefill_qk_l2norm"] = {
+            "metric": "prefill tokens/s with in-kernel q/k L2 normalisation (same workload)",
+            "value": round(dist.world * tokens / (l_ms / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(l_ms, 4),
+            "roofline": {"bound": "hbm", "frac": round(algo_bytes / (l_ms / 1e3) / 1e9 / hbm_peak, 4),
+                         "peak": hbm_peak, "unit": "GB/s", "peak_kind": peak_kind},
+        }
         secondary["decode"] = bench_decode(dev, dist, stream, hbm_peak, peak_kind)
         secondary["varlen"] = bench_varlen(dev, dist, stream, flush, hbm_peak, peak_kind)
     clk = clocks.stop()

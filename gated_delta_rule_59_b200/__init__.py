@@ -48,10 +48,12 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         vp, fp, ip, i32 = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32
         L.dr_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i32, i32, i32, i32, i32, i32,
-                                   ctypes.c_int, ctypes.c_float, vp, ctypes.c_int, fp, vp]
+                                   ctypes.c_int, ctypes.c_float, vp, ctypes.c_int, fp,
+                                   ctypes.c_uint32, vp]
         L.dr_chunk_fwd.restype = ctypes.c_int
         L.dr_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, i32,
-                                        ctypes.c_int, ctypes.c_float, vp, ctypes.c_int, vp]
+                                        ctypes.c_int, ctypes.c_float, vp, ctypes.c_int,
+                                        ctypes.c_uint32, vp]
         L.dr_recurrent_step.restype = ctypes.c_int
         L.dr_status_string.argtypes = [ctypes.c_int]
         L.dr_status_string.restype = ctypes.c_char_p
@@ -93,12 +95,14 @@ def _stream(device) -> ctypes.c_void_p:
 
 
 def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
-              output_final_state: bool = True, out_dtype=torch.float32, o=None, state_out=None):
+              output_final_state: bool = True, out_dtype=torch.float32, o=None, state_out=None,
+              qk_l2norm: bool = False):
     """Chunked prefill through ``dr_chunk_fwd``.
 
     q, k [B, T, Hqk, dk] and v [B, T, Hv, dv] in bf16 or fp32 (same dtype);
     g (or None), beta [B, T, Hv] fp32; state_in [N, Hv, dk, dv] fp32 or None;
-    cu_seqlens int32 [N+1] (device) or None.  Returns (o [B, T, Hv, dv] in
+    cu_seqlens int32 [N+1] (device) or None.  ``qk_l2norm``: the kernel divides every q and
+    k row by its L2 norm first (``DR_QK_L2NORM``).  Returns (o [B, T, Hv, dv] in
     ``out_dtype``, state_out [N, Hv, dk, dv] fp32 or None).
     """
     if q.dtype not in _DTYPES or out_dtype not in _DTYPES:
@@ -129,17 +133,19 @@ def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1
     rc = lib().dr_chunk_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), N,
         B, T, Hqk, Hv, dk, dv, _DTYPES[q.dtype], float(scale), _ptr(o), _DTYPES[out_dtype],
-        _ptr(state_out), _stream(dev))
+        _ptr(state_out), QK_L2NORM if qk_l2norm else 0, _stream(dev))
     if rc != 0:
         raise DrError(rc, "dr_chunk_fwd")
     return o, state_out
 
 
-def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.float32, o=None):
+def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.float32, o=None,
+                   qk_l2norm: bool = False):
     """One decode step through ``dr_recurrent_step``; ``state`` is updated in place.
 
     q, k [B, Hqk, dk], v [B, Hv, dv] (bf16 or fp32); g (or None), beta [B, Hv] fp32;
-    state [B, Hv, dk, dv] fp32.  Returns o [B, Hv, dv] in ``out_dtype``.
+    state [B, Hv, dk, dv] fp32.  ``qk_l2norm`` as for ``chunk_fwd``.  Returns o [B, Hv, dv] in
+    ``out_dtype``.
     """
     if q.dtype not in _DTYPES or out_dtype not in _DTYPES:
         raise ValueError("q/k/v must be bf16 or fp32; out_dtype bf16 or fp32")
@@ -157,13 +163,15 @@ def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.
     _check(o, "o", out_dtype, dev)
     rc = lib().dr_recurrent_step(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), B, Hqk, Hv, dk, dv,
-        _DTYPES[q.dtype], float(scale), _ptr(o), _DTYPES[out_dtype], _stream(dev))
+        _DTYPES[q.dtype], float(scale), _ptr(o), _DTYPES[out_dtype],
+        QK_L2NORM if qk_l2norm else 0, _stream(dev))
     if rc != 0:
         raise DrError(rc, "dr_recurrent_step")
     return o
 
 
 KERNELS = {0: None, 1: "simt_f32", 2: "tc_bf16"}
+QK_L2NORM = 1  # DR_QK_L2NORM of include/dr.h
 
 
 def prefill_kernel(dtype, dk: int, dv: int):

@@ -147,6 +147,28 @@ __device__ __forceinline__ void chunk_gates(const PrefillArgs &a, float *gs, int
   }
 }
 
+// Sum of squares of row r of a 64 x 128 bf16 operand held as two 128-byte-swizzled boxes of
+// 64 columns (box0, box0 + 16384), e.g. one K or Q tile of a chunk.
+__device__ __forceinline__ float row_sumsq(uint32_t box0, int r) {
+  float acc = 0.f;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 w = tc::ld_shared_v4(box0 + 16384u * b + tc::sw128_off(r, j));
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float lo = __uint_as_float(ws[t] << 16), hi = __uint_as_float(ws[t] & 0xffff0000u);
+        acc = fmaf(lo, lo, acc);
+        acc = fmaf(hi, hi, acc);
+      }
+    }
+  }
+  return acc;
+}
+__device__ __forceinline__ float inv_norm(float sumsq) { return sumsq > 0.f ? rsqrtf(sumsq) : 0.f; }
+
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
   const float h0 = __bfloat162float(__float2bfloat16_rn(x0));
   const float h1 = __bfloat162float(__float2bfloat16_rn(x1));
@@ -154,7 +176,9 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_
   lo = tc::pack_bf16(x0 - h0, x1 - h1);
 }
 
-template <bool OUT_F32>
+// L2N: q and k rows are L2-normalised first (a compile-time switch, so that the plain path
+// carries none of its code).
+template <bool OUT_F32, bool L2N>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -334,12 +358,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
       const int pi = wg - 1, pt = tid - 128 * wg;  // pt: 0..127
       const uint32_t nb = 1 + (uint32_t)pi;        // named barrier of the instance (128)
       const uint32_t nbL = 3 + (uint32_t)pi;       // named barrier of its two L warps (64)
+      const uint32_t nbP = 5 + (uint32_t)pi;       // named barrier of its two P warps (64)
       const uint32_t wa = sb + P_OFF_WA + (uint32_t)pi * WA_BYTES;
       float *LT = reinterpret_cast<float *>(smem + P_OFF_WA + pi * WA_BYTES + WA_LT);
       float *Tf = reinterpret_cast<float *>(smem + P_OFF_TF + pi * TF_BYTES);  // T, row-major
       float *Xs = reinterpret_cast<float *>(smem + P_OFF_WA + pi * WA_BYTES + WA_X);  // scratch
       float *TDT = Xs + 512;  // diagonal blocks of T transposed [4][16 m][16 r]
-      const float *gs = reinterpret_cast<const float *>(smem + P_OFF_GATES) + 192 * pi;
+      float *gsm = reinterpret_cast<float *>(smem + P_OFF_GATES) + 192 * pi;
+      const float *gs = gsm;
       const uint32_t colG = 128u * (uint32_t)pi, colW = colG + 64;
       // G rows 0-63 are K K^T for instance 0 and Q K^T for instance 1: the warps on the
       // TMEM lanes of the K K^T rows build L and T, the other two build P.
@@ -354,16 +380,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         }
         role_wait(P_G_FULL + pi, ph, pt == 0, nb, 128);
         tc::tc_fence_after();
+        // this thread's row of G: a row of K K^T (L warps) or of Q K^T (P warps)
+        uint32_t u0[32], u1[32];
+        tc::tmem_ld32_nw(tmem + lane_off + colG, u0);
+        tc::tmem_ld32_nw(tmem + lane_off + colG + 32, u1);
+        tc::tmem_wait_ld();
+        tc::reg_fence(u0);
+        tc::reg_fence(u1);
+        // q/k L2 normalisation as exact fp32 scalings: L and P take 1/|k_s| per column and
+        // 1/|k_r| or 1/|q_r| per row; T diag(beta gamma) takes 1/|k_s| per column (W = T
+        // diag(beta gamma) K^).  |k_r|^2 is the diagonal of K K^T; the column factors are
+        // exchanged through the diagonal of L^T, which is never read as L.
+        float rinv = 1.f;
+        if constexpr (L2N) {
+          if (lrole) {
+            float d = 0.f;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              if (t == rr) d = __uint_as_float(u0[t]);
+              if (t + 32 == rr) d = __uint_as_float(u1[t]);
+            }
+            rinv = inv_norm(d);
+            LT[rr * 65] = rinv;
+            gsm[128 + rr] *= rinv;
+          } else {
+            if (rr == 0) wait(P_KQ_FULL + (c % (int)P_NKQ), ((uint32_t)c / P_NKQ) & 1u);
+            tc::named_bar(nbP, 64);  // the Q tile of this chunk is visible to every P thread
+            const uint32_t qbox = sb + ((uint32_t)c % P_NKQ) * KQ_BYTES + ((c & 1) ? 0u : 8192u);
+            rinv = inv_norm(row_sumsq(qbox, rr));
+          }
+          tc::named_bar(nb, 128);  // every 1/|k_s| is on the diagonal of L^T
+        }
         if (lrole) {
           // ---- L^T[s][r] = L_rs = beta_r Gamma_rs (k_r . k_s), s < r; r = this thread ----
           {
-            uint32_t u0[32], u1[32];
-            tc::tmem_ld32_nw(tmem + lane_off + colG, u0);
-            tc::tmem_ld32_nw(tmem + lane_off + colG + 32, u1);
-            const float br = gs[rr], bt = gs[64 + rr];
-            tc::tmem_wait_ld();
-            tc::reg_fence(u0);
-            tc::reg_fence(u1);
+            const float br = gs[rr], bt = gs[64 + rr] * rinv;
 #pragma unroll
             for (int q = 0; q < 16; ++q) {
               const float4 b4 = reinterpret_cast<const float4 *>(gs)[q];
@@ -372,7 +423,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
               for (int t = 0; t < 4; ++t) {
                 const int s_ = 4 * q + t;
                 const float kk = __uint_as_float(s_ < 32 ? u0[s_ & 31] : u1[s_ & 31]);
-                LT[s_ * 64 + rr] = (s_ < rr) ? bt * tc::ex2(br - bs[t]) * kk : 0.f;
+                const float cs = L2N ? LT[s_ * 65] : 1.f;
+                LT[s_ * 64 + rr] = (s_ < rr) ? bt * tc::ex2(br - bs[t]) * kk * cs
+                                             : ((s_ == rr && L2N) ? rinv : 0.f);
               }
             }
           }
@@ -400,13 +453,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           }
         } else {
           // ---- P rows: scale Gamma_rs (q_r . k_s), s <= r -> bf16 hi/lo tiles ----
-          uint32_t u0[32], u1[32];
-          tc::tmem_ld32_nw(tmem + lane_off + colG, u0);
-          tc::tmem_ld32_nw(tmem + lane_off + colG + 32, u1);
-          const float br = gs[rr];
-          tc::tmem_wait_ld();
-          tc::reg_fence(u0);
-          tc::reg_fence(u1);
+          const float br = gs[rr], sr = a.scale * rinv;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const float4 b4a = reinterpret_cast<const float4 *>(gs)[2 * q];
@@ -417,7 +464,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
             for (int t = 0; t < 8; ++t) {
               const int s_ = 8 * q + t;
               const float qk = __uint_as_float(s_ < 32 ? u0[s_ & 31] : u1[s_ & 31]);
-              v[t] = (s_ <= rr) ? a.scale * tc::ex2(br - bs[t]) * qk : 0.f;
+              const float cs = L2N ? LT[s_ * 65] : 1.f;
+              v[t] = (s_ <= rr) ? sr * tc::ex2(br - bs[t]) * qk * cs : 0.f;
             }
             tck::st_row_chunk_split(wa + WA_T, wa + WA_T + 8192, rr, q, v);
           }
@@ -604,8 +652,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           if (lane == 0) wait_sleep(S_GATE_EMPTY + s, ((uint32_t)(c - 2) >> 1) & 1u);
           __syncwarp();
         }
-        chunk_gates(a, reinterpret_cast<float *>(smem + S_OFF_GATES) + 256 * s, zbase, t0,
-                    min(C, eos - t0), h, lane, true);
+        float *gsl = reinterpret_cast<float *>(smem + S_OFF_GATES) + 256 * s;
+        chunk_gates(a, gsl, zbase, t0, min(C, eos - t0), h, lane, true);
+        // the output scaling gam_r (/ |q_r|) goes to the first array (bs2 is not used here);
+        // the state update's e^{b_C - b_s} takes 1/|k_s|
+        if constexpr (L2N) {
+          if (lane == 0) wait(S_QK_FULL + s, ((uint32_t)c >> 1) & 1u);
+          __syncwarp();
+          const uint32_t stg = sb + S_OFF_QK + (uint32_t)s * KQ_BYTES;
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = lane + 32 * hh;
+            gsl[192 + r] *= inv_norm(row_sumsq(stg + KQ_K0, r));
+            gsl[r] = gsl[128 + r] * inv_norm(row_sumsq(stg + KQ_Q0, r));
+          }
+        } else {
+          gsl[lane] = gsl[128 + lane];
+          gsl[lane + 32] = gsl[160 + lane];
+        }
         tck::warp_arrive(bar(S_GATE_FULL + s), lane);
       }
     } else if (warp == 3) {
@@ -729,7 +793,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
           }
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float4 g4 = reinterpret_cast<const float4 *>(gs + 128 + 32 * half)[q];
+            const float4 g4 = reinterpret_cast<const float4 *>(gs + 32 * half)[q];
             const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
             for (int t = 0; t < 4; ++t)
@@ -780,7 +844,10 @@ inline cudaError_t pair_dispatch(bool out_f32, const PrefillArgs &a, int N, cuda
       !tck::make_map(&mv, a.v, 128, a.Hv, rows) ||
       !tck::make_map_out(&mo, a.o, 128, a.Hv, rows, out_f32))
     return cudaErrorInvalidValue;
-  auto kern = out_f32 ? tcp::chunk_pair_kernel<true> : tcp::chunk_pair_kernel<false>;
+  auto kern = out_f32 ? (a.qk_l2norm ? tcp::chunk_pair_kernel<true, true>
+                                     : tcp::chunk_pair_kernel<true, false>)
+                      : (a.qk_l2norm ? tcp::chunk_pair_kernel<false, true>
+                                     : tcp::chunk_pair_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcp::SMEM_BYTES);
   if (e != cudaSuccess) return e;

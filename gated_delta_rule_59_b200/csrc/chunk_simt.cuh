@@ -33,6 +33,7 @@ struct PrefillArgs {
   float scale;
   void *o;
   float *state_out;
+  int qk_l2norm;  // 1: divide q and k rows by their L2 norms first (zero rows stay zero)
 };
 
 template <int DK, int DVS, int C>
@@ -98,6 +99,25 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(PrefillArgs a, int dv) 
     for (int idx = tid; idx < C * DVS; idx += NT) {
       const int r = idx / DVS, j = idx % DVS;
       Vs[r * VP + j] = r < L ? io<Tin>::ld(v + (((size_t)batch * a.T + c0 + r) * a.Hv + h) * dv + j0 + j) : 0.f;
+    }
+    if (a.qk_l2norm) {  // rows of K and of Q (= scale q) divided by their norms
+      __syncthreads();
+      const int w = tid >> 5, ln = tid & 31;
+      for (int r = w; r < C; r += NT / 32) {
+        float sk = 0.f, sq = 0.f;
+        for (int i = ln; i < DK; i += 32) {
+          sk += Ks[r * KP + i] * Ks[r * KP + i];
+          sq += Qs[r * KP + i] * Qs[r * KP + i];
+        }
+        sk = warp_sum(sk);
+        sq = warp_sum(sq);
+        const float ik = sk > 0.f ? rsqrtf(sk) : 0.f;
+        const float iq = sq > 0.f ? fabsf(a.scale) * rsqrtf(sq) : 0.f;  // |scale| / |scale q|
+        for (int i = ln; i < DK; i += 32) {
+          Ks[r * KP + i] *= ik;
+          Qs[r * KP + i] *= iq;
+        }
+      }
     }
     if (tid < 32) {
       // inclusive prefix sum of g over the chunk (C <= 32 handled per lane)

@@ -35,12 +35,12 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
     decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                        const Tin *__restrict__ v, const float *__restrict__ g,
                        const float *__restrict__ beta, float *__restrict__ state, int Hqk,
-                       int Hv, float scale, Tout *__restrict__ o) {
+                       int Hv, float scale, Tout *__restrict__ o, int l2n) {
   using S = DecodeShape<DK, DV>;
   constexpr int C4 = S::C4, RP = S::RP, NT = S::NT, RPT = S::RPT;
   __shared__ float ks[DK], qs[DK];
   __shared__ float4 red_k[RP][C4], red_q[RP][C4];
-  __shared__ float qk_shared;
+  __shared__ float qk_shared, nrm[2];
 
   const int unit = blockIdx.x;  // b * Hv + h
   const int b = unit / Hv, h = unit - (unit / Hv) * Hv;
@@ -59,6 +59,23 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
     qs[i] = scale * io<Tin>::ld(q + qk_off + i);
   }
   __syncthreads();
+  if (l2n) {  // k and q (= scale q) rows divided by their norms; zero rows stay zero
+    if (t < 64) {
+      const float *x = (t < 32) ? ks : qs;
+      float acc = 0.f;
+      for (int i = t & 31; i < DK; i += 32) acc += x[i] * x[i];
+      acc = warp_sum(acc);
+      if ((t & 31) == 0)
+        nrm[t >> 5] = acc > 0.f ? ((t < 32) ? rsqrtf(acc) : fabsf(scale) * rsqrtf(acc)) : 0.f;
+    }
+    __syncthreads();
+    const float ik = nrm[0], iq = nrm[1];
+    for (int i = t; i < DK; i += NT) {
+      ks[i] *= ik;
+      qs[i] *= iq;
+    }
+    __syncthreads();
+  }
   if (t < 32) {
     float acc = 0.f;
     for (int i = t; i < DK; i += 32) acc += ks[i] * qs[i];
@@ -112,10 +129,11 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
 template <int DK, int DV, typename Tin, typename Tout>
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *state, int B, int Hqk, int Hv, float scale,
-                          void *o, cudaStream_t stream) {
+                          void *o, int l2n, cudaStream_t stream) {
   const unsigned units = (unsigned)B * (unsigned)Hv;
   decode_step_kernel<DK, DV, Tin, Tout><<<units, DecodeShape<DK, DV>::NT, 0, stream>>>(
-      (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, Hqk, Hv, scale, (Tout *)o);
+      (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, Hqk, Hv, scale, (Tout *)o,
+      l2n);
   return cudaGetLastError();
 }
 

@@ -25,10 +25,11 @@ bool dtype_ok(dr_dtype t) { return t == DR_F32 || t == DR_BF16; }
 template <typename Tin, typename Tout>
 cudaError_t decode_dispatch(int dk, int dv, const void *q, const void *k, const void *v,
                             const float *g, const float *beta, float *state, int B, int Hqk,
-                            int Hv, float scale, void *o, cudaStream_t s) {
+                            int Hv, float scale, void *o, int l2n, cudaStream_t s) {
 #define DR_DEC(DK, DV)                                                                  \
   if (dk == DK && dv == DV)                                                             \
-    return dr::launch_decode<DK, DV, Tin, Tout>(q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s);
+    return dr::launch_decode<DK, DV, Tin, Tout>(q, k, v, g, beta, state, B, Hqk, Hv, scale, o, \
+                                                l2n, s);
 #define DR_DEC_ROW(DK) DR_DEC(DK, 16) DR_DEC(DK, 32) DR_DEC(DK, 64) DR_DEC(DK, 128)
   DR_DEC_ROW(16) DR_DEC_ROW(32) DR_DEC_ROW(64) DR_DEC_ROW(128)
 #undef DR_DEC_ROW
@@ -62,8 +63,9 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
                        const float *beta, const float *state_in, const int32_t *cu_seqlens,
                        int32_t n_seqs, int32_t B, int32_t T, int32_t Hqk, int32_t Hv,
                        int32_t dk, int32_t dv, dr_dtype in_dtype, float scale, void *o,
-                       dr_dtype o_dtype, float *state_out, dr_stream stream) {
+                       dr_dtype o_dtype, float *state_out, uint32_t flags, dr_stream stream) {
   if (!dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return DR_ERR_DTYPE;
+  if (flags & ~DR_QK_L2NORM) return DR_ERR_UNSUPPORTED;
   if (B < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return DR_ERR_SHAPE;
   if (Hv % Hqk != 0) return DR_ERR_SHAPE;
   if (cu_seqlens && (B != 1 || n_seqs < 0)) return DR_ERR_SHAPE;
@@ -81,7 +83,7 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   dr::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, (int)N, B, T, Hqk, Hv,
-                    scale, o, state_out};
+                    scale, o, state_out, (flags & DR_QK_L2NORM) ? 1 : 0};
   cudaError_t e;
   if (in_dtype == DR_BF16 && dr::tc_supported(dk, dv)) {
     e = dr::prefill_tc_dispatch(dk, dv, o_dtype == DR_F32, a, (int)N, s);
@@ -96,8 +98,10 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
 dr_status dr_recurrent_step(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, float *state, int32_t B, int32_t Hqk,
                             int32_t Hv, int32_t dk, int32_t dv, dr_dtype in_dtype,
-                            float scale, void *o, dr_dtype o_dtype, dr_stream stream) {
+                            float scale, void *o, dr_dtype o_dtype, uint32_t flags,
+                            dr_stream stream) {
   if (!dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return DR_ERR_DTYPE;
+  if (flags & ~DR_QK_L2NORM) return DR_ERR_UNSUPPORTED;
   if (B < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return DR_ERR_SHAPE;
   if (Hv % Hqk != 0) return DR_ERR_SHAPE;
   if (!dim_ok(dk) || !dim_ok(dv)) return DR_ERR_UNSUPPORTED;
@@ -109,15 +113,16 @@ dr_status dr_recurrent_step(const void *q, const void *k, const void *v, const f
     return DR_ERR_ALIGN;
   if ((int64_t)B * Hv > 0x7fffffff) return DR_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int l2n = (flags & DR_QK_L2NORM) ? 1 : 0;
   cudaError_t e;
   if (in_dtype == DR_BF16)
     e = o_dtype == DR_F32
-            ? decode_dispatch<__nv_bfloat16, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s)
-            : decode_dispatch<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s);
+            ? decode_dispatch<__nv_bfloat16, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, s)
+            : decode_dispatch<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, s);
   else
     e = o_dtype == DR_F32
-            ? decode_dispatch<float, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s)
-            : decode_dispatch<float, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, s);
+            ? decode_dispatch<float, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, s)
+            : decode_dispatch<float, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, s);
   return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 

@@ -63,13 +63,20 @@ typedef enum { DR_F32 = 0, DR_BF16 = 1 } dr_dtype;
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st *dr_stream;
 
+/* Option bits of dr_chunk_fwd / dr_recurrent_step (any other bit => DR_ERR_UNSUPPORTED). */
+#define DR_QK_L2NORM 1u /* divide every q and k row (per token and q/k head) by its L2 norm
+                           first (an all-zero row stays zero): the pages' qk_l2norm step
+                           ("DeltaNet Attention": queries and keys are L2-normalised before
+                           the rule), folded into the kernels as fp32 row and column scalings */
+
 /*
  * dr_chunk_fwd -- prompt (prefill) pass: the "chunked rule on a prompt" of the
  * "linear_attention" page, computed chunkwise in the UT/WY form of
  * "Parallelizing Linear Transformers with the Delta Rule over Sequence Length"
  * (the reference both DeltaNet pages cite), 64-token chunks, decays folded in.
  *
- *   q, k       [B, T, Hqk, dk]   in_dtype (DR_BF16 or DR_F32), L2-normalised by the caller
+ *   q, k       [B, T, Hqk, dk]   in_dtype (DR_BF16 or DR_F32); L2-normalised by the caller,
+ *                                or by the kernel with DR_QK_L2NORM in flags
  *   v          [B, T, Hv, dv]    in_dtype
  *   g          [B, T, Hv] f32    log decay (<= 0 expected); NULL => no decay (plain DeltaNet)
  *   beta       [B, T, Hv] f32    write strength
@@ -82,6 +89,7 @@ typedef struct CUstream_st *dr_stream;
  *   o          [B, T, Hv, dv]    o_dtype (DR_F32 or DR_BF16); every token's output is written
  *   state_out  [N, Hv, dk, dv] f32 or NULL (=> final state not returned).  It may be
  *              state_in itself (in-place update); a partial overlap is undefined.
+ *   flags      0 or DR_QK_L2NORM
  *   T = 0 or N = 0 is valid: nothing is read from q/k/v; state_out (if given) receives
  *   state_in (or zeros).
  */
@@ -90,7 +98,7 @@ DR_API dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const
                               const int32_t *cu_seqlens, int32_t n_seqs, int32_t B, int32_t T,
                               int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv,
                               dr_dtype in_dtype, float scale, void *o, dr_dtype o_dtype,
-                              float *state_out, dr_stream stream);
+                              float *state_out, uint32_t flags, dr_stream stream);
 
 /* Which prefill kernel dr_chunk_fwd launches for these inputs (host only, no device call). */
 typedef enum {
@@ -117,7 +125,7 @@ DR_API dr_status dr_recurrent_step(const void *q, const void *k, const void *v,
                                    const float *g, const float *beta, float *state, int32_t B,
                                    int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv,
                                    dr_dtype in_dtype, float scale, void *o, dr_dtype o_dtype,
-                                   dr_stream stream);
+                                   uint32_t flags, dr_stream stream);
 
 /* Static English description of a status code (never NULL). */
 DR_API const char *dr_status_string(dr_status status);

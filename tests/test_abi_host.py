@@ -55,15 +55,15 @@ P4 = ctypes.c_void_p(0x10004)
 
 
 def chunk(L, q=P16, k=P16, v=P16, g=None, beta=P16, s_in=None, cu=None, n_seqs=0, B=1, T=8,
-          Hqk=1, Hv=1, dk=64, dv=64, dt=1, scale=1.0, o=P16, odt=0, s_out=None):
+          Hqk=1, Hv=1, dk=64, dv=64, dt=1, scale=1.0, o=P16, odt=0, s_out=None, flags=0):
     return L.dr_chunk_fwd(q, k, v, g, beta, s_in, cu, n_seqs, B, T, Hqk, Hv, dk, dv, dt, scale,
-                          o, odt, s_out, None)
+                          o, odt, s_out, flags, None)
 
 
 def step(L, q=P16, k=P16, v=P16, g=None, beta=P16, state=P16, B=2, Hqk=1, Hv=1, dk=64, dv=64,
-         dt=1, scale=1.0, o=P16, odt=0):
+         dt=1, scale=1.0, o=P16, odt=0, flags=0):
     return L.dr_recurrent_step(q, k, v, g, beta, state, B, Hqk, Hv, dk, dv, dt, scale, o, odt,
-                               None)
+                               flags, None)
 
 
 def test_chunk_fwd_argument_errors(L):
@@ -83,6 +83,10 @@ def test_chunk_fwd_argument_errors(L):
     assert chunk(L, q=ctypes.c_void_p(0x10008)) == 4
     assert chunk(L, s_in=ctypes.c_void_p(0x10004)) == 4
     assert chunk(L, g=ctypes.c_void_p(0x10002)) == 4
+    # option bits: DR_QK_L2NORM (1) is known, any other bit is unsupported
+    assert chunk(L, flags=2) == 5
+    assert chunk(L, flags=0x80000001) == 5
+    assert chunk(L, B=0, flags=1) == 0
     # nothing to do: no sequences => OK without touching the device
     assert chunk(L, B=0) == 0
     assert chunk(L, cu=P16, n_seqs=0) == 0
@@ -99,6 +103,8 @@ def test_recurrent_step_argument_errors(L):
     assert step(L, v=None) == 1
     assert step(L, o=ctypes.c_void_p(0x10004)) == 4
     assert step(L, g=ctypes.c_void_p(0x10001)) == 4
+    assert step(L, flags=4) == 5
+    assert step(L, B=0, flags=1) == 0
     assert step(L, B=0) == 0
 
 

@@ -80,3 +80,34 @@ def test_decode_bf16_output(cuda_device):
         # bf16 storage of the output adds at most half an ulp (2^-8 relative) per element
         err = np.abs(to64(o) - r) - 2.0 ** -8 * np.abs(r)
         assert np.max(err) / np.sqrt(np.mean(r ** 2)) <= TOL_BF16
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_decode_qk_l2norm_option(cuda_device, dtype):
+    """DR_QK_L2NORM on decode: rescaled q/k rows (one all-zero k) normalised in the kernel."""
+    state0, steps = inputs.decode_config(n_steps=4, B=16)
+    gen = torch.Generator().manual_seed(5)
+    new = []
+    for i, s in enumerate(steps):
+        cq = torch.empty(s.q.shape[:-1] + (1,)).uniform_(0.2, 5.0, generator=gen)
+        ck = torch.empty(s.k.shape[:-1] + (1,)).uniform_(0.2, 5.0, generator=gen)
+        q = (s.q.float() * cq).to(dtype)
+        k = (s.k.float() * ck).to(dtype)
+        if i == 1:
+            k[3] = 0.0
+        new.append(inputs.DecodeStep(q.contiguous(), k.contiguous(), s.v.to(dtype), s.g, s.beta))
+    state = state0.to(cuda_device).contiguous()
+    outs = []
+    for s in new:
+        d = s.to(cuda_device)
+        outs.append(dr.recurrent_step(d.q, d.k, d.v, d.g, d.beta, state, scale=0.125,
+                                      qk_l2norm=True).cpu())
+    torch.cuda.synchronize()
+    assert dr.device_status() == 0
+    st = to64(state0)
+    for s, o in zip(new, outs):
+        ro, st = oracle.step(s.q, s.k, s.v, s.g, s.beta, st, scale=0.125, qk_l2norm=True)
+        metric, tol = metric_for(dtype)
+        assert metric(o, ro) <= tol
+    metric, tol = metric_for(dtype)
+    assert metric(state.cpu(), st) <= tol

@@ -54,6 +54,39 @@ def test_head_dims(cuda_device, dk, dv, dtype):
     check_full(p, cuda_device, scale=dk ** -0.5)
 
 
+def _rescaled_rows(x, seed, zero_token=None):
+    """Rows (last axis) multiplied by random positive factors, one token zeroed; same dtype."""
+    gen = torch.Generator().manual_seed(seed)
+    c = torch.empty(x.shape[:-1] + (1,)).uniform_(0.2, 5.0, generator=gen)
+    y = x.float() * c
+    if zero_token is not None:
+        y[:, zero_token] = 0.0
+    return y.to(x.dtype).contiguous()
+
+
+@pytest.mark.parametrize("dtype,d,T,group", [(torch.bfloat16, 128, 200, 2),
+                                             (torch.bfloat16, 128, 64, 1),
+                                             (torch.bfloat16, 64, 130, 2),
+                                             (torch.float32, 64, 97, 1)])
+def test_qk_l2norm_option(cuda_device, dtype, d, T, group):
+    """DR_QK_L2NORM: q/k rows rescaled (one token all zero) and normalised by the kernel,
+    against the oracle normalising the same inputs in fp64; scale = d^-1/2."""
+    p = inputs.prefill(2, T, 2, 2 * group, d, d, dtype, gated=True, state_std=0.02,
+                       seed=300 + T + d)
+    q = _rescaled_rows(p.q, 1, zero_token=T // 3)
+    k = _rescaled_rows(p.k, 2, zero_token=T // 2)
+    scale = d ** -0.5
+    dev = cuda_device
+    o, st = dr.chunk_fwd(q.to(dev), k.to(dev), p.v.to(dev), p.g.to(dev), p.beta.to(dev),
+                         p.state_in.to(dev), None, scale=scale, qk_l2norm=True)
+    torch.cuda.synchronize()
+    assert dr.device_status() == 0
+    ro, rs = oracle.run(q, k, p.v, p.g, p.beta, p.state_in, None, scale=scale, qk_l2norm=True)
+    metric, tol = metric_for(dtype)
+    eo, es = metric(o.cpu(), ro), metric(st.cpu(), rs)
+    assert eo <= tol and es <= tol, (eo, es)
+
+
 def test_many_units_several_cluster_waves(cuda_device):
     """B=3, Hv=32: 96 (sequence, head) units = 192 CTAs of 2-CTA clusters, more than one wave
     on 148 SMs; every output and final state against the oracle."""
