@@ -237,9 +237,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
   const uint32_t tmem = *tmem_slot;
 
   auto wait = [&](int i, uint32_t parity) { tc::mbar_wait(bar(i), parity, abort_flag); };
-  auto wait_sleep = [&](int i, uint32_t parity) {
-    tc::mbar_wait_sleep(bar(i), parity, abort_flag);
-  };
+  // Producers and gates poll too: a thread suspended in try_wait was measured to resume up to
+  // ~1 us after the phase completed, and the gates of a chunk are on its instance's path.
+  auto wait_sleep = [&](int i, uint32_t parity) { tc::mbar_wait(bar(i), parity, abort_flag); };
   // Phases completed from the partner CTA are polled at CTA scope too: incoming operands are
   // made visible by the copies' complete_tx (as for any bulk or TMA copy), and the partner's
   // acknowledgements publish no data.  (Cluster-scope acquire polls measured slower.)
