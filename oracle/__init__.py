@@ -55,7 +55,7 @@ def _load():
             dp, dp, dp, dp, dp, dp, ip,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int,
-            dp, dp,
+            dp, dp, ctypes.c_int, dp,
         ]
         lib.oracle_run.restype = ctypes.c_int
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -94,14 +94,37 @@ def l2_normalize_rows(x):
     return np.where(n > 0.0, x / np.where(n > 0.0, n, 1.0), 0.0)
 
 
+def chunk_rows(cu_seqlens, B: int, T: int, chunk_len: int):
+    """First chunk-state row of every sequence and the total row count.
+
+    Sequence n owns ceil(len_n / chunk_len) rows, in sequence order; a sequence of length
+    zero owns none.  Returns (bases [N] as a list of ints, total).
+    """
+    if cu_seqlens is None:
+        lens = [T] * B
+    else:
+        cu = [int(x) for x in np.asarray(cu_seqlens)]
+        lens = [cu[n + 1] - cu[n] for n in range(len(cu) - 1)]
+    bases, tot = [], 0
+    for ln in lens:
+        bases.append(tot)
+        tot += -(-ln // chunk_len)
+    return bases, tot
+
+
 def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
-        form: int = 2, threads: int = 0, qk_l2norm: bool = False):
+        form: int = 2, threads: int = 0, qk_l2norm: bool = False, chunk_len: int = 0):
     """Token-by-token fp64 recurrence.
 
     q, k: [B, T, Hqk, dk]; v: [B, T, Hv, dv]; g, beta: [B, T, Hv] (g may be None);
     state_in: [N, Hv, dk, dv] or None (zeros); cu_seqlens: int [N+1] or None.
     ``qk_l2norm``: q and k rows are L2-normalised first (``l2_normalize_rows``).
     Returns (o [B, T, Hv, dv], state_out [N, Hv, dk, dv]) as float64 numpy arrays.
+    With ``chunk_len`` > 0 a third array is returned: the stored state after every
+    ``chunk_len`` tokens of each sequence and after its last token,
+    [sum_n ceil(len_n / chunk_len), Hv, dk, dv], rows ordered as ``chunk_rows`` gives.
+    This is the intermediate state the "DeltaNet" tracing route exposes (the state after
+    every token, of which these are the chunk-boundary samples).
     """
     lib = _load()
     q, k, v, g, beta, state_in = (_f64(a) for a in (q, k, v, g, beta, state_in))
@@ -124,14 +147,17 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
         assert state_in.shape == (N, Hv, dk, dv), state_in.shape
     o = np.zeros((B, T, Hv, dv), dtype=np.float64)
     st = np.zeros((N, Hv, dk, dv), dtype=np.float64)
+    cs = None
+    if chunk_len > 0:
+        cs = np.zeros((chunk_rows(cu, B, T, chunk_len)[1], Hv, dk, dv), dtype=np.float64)
     rc = lib.oracle_run(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
         _ptr(cu, ctypes.c_int32), N, B, T, Hqk, Hv, dk, dv, float(scale), int(form),
-        int(threads), _ptr(o), _ptr(st),
+        int(threads), _ptr(o), _ptr(st), int(chunk_len), _ptr(cs),
     )
     if rc != 0:
         raise ValueError(f"oracle_run failed with code {rc}")
-    return o, st
+    return (o, st) if cs is None else (o, st, cs)
 
 
 def step(q, k, v, g, beta, state, scale: float = 1.0, form: int = 2, threads: int = 0,

@@ -47,11 +47,14 @@ def chunk_step(Q, K, V, g, beta, H0):
     return O, H1
 
 
-def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale=1.0, chunk=64):
+def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale=1.0, chunk=64,
+        chunk_states=False):
     """Chunk form over a whole (possibly varlen-packed) batch.
 
     Same layouts and return values as ``oracle.run``.  The last chunk of a
-    sequence may be shorter than ``chunk``.
+    sequence may be shorter than ``chunk``.  With ``chunk_states`` a third array
+    holds H_L of every chunk, sequence after sequence (the rows ``oracle.run`` with
+    ``chunk_len=chunk`` returns).
     """
     q, k, v, beta = (np.asarray(a, dtype=np.float64) for a in (q, k, v, beta))
     B, T, Hqk, dk = q.shape
@@ -66,6 +69,8 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale=1.0, chunk=64):
     group = Hv // Hqk
     o = np.zeros((B, T, Hv, dv))
     st = np.zeros((N, Hv, dk, dv))
+    rows = [(n, c0) for n, (bb, t0, t1) in enumerate(seqs) for c0 in range(t0, t1, chunk)]
+    cs = np.zeros((len(rows), Hv, dk, dv))
     for n, (bb, t0, t1) in enumerate(seqs):
         for h in range(Hv):
             hq = h // group
@@ -75,5 +80,6 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale=1.0, chunk=64):
                 O, H = chunk_step(scale * q[bb, c0:c1, hq], k[bb, c0:c1, hq], v[bb, c0:c1, h],
                                   g[bb, c0:c1, h], beta[bb, c0:c1, h], H)
                 o[bb, c0:c1, h] = O
+                cs[rows.index((n, c0)), h] = H
             st[n, h] = H
-    return o, st
+    return (o, st, cs) if chunk_states else (o, st)

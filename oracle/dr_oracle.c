@@ -105,6 +105,12 @@ static void update_form3(double *S, const double *k, const double *v, double alp
  *   g, beta     [B, T, Hv]        (g may be NULL: no decay)
  *   state_in    [N, Hv, dk, dv]   (may be NULL: zero state)
  *   state_out   [N, Hv, dk, dv]   (may be NULL)
+ *   chunk_states [NC, Hv, dk, dv] (may be NULL): the stored state S^T after
+ *                every chunk_len tokens of each sequence and after its last
+ *                token.  Sequence n owns ceil(len_n / chunk_len) rows starting
+ *                at the sum of that count over the sequences before it; row j
+ *                holds the state after min((j+1) chunk_len, len_n) tokens, so a
+ *                sequence's last row equals its state_out.
  * With cu_seqlens (host int32 [N+1], N = n_seqs) B must be 1 and sequence n
  * covers tokens [cu_seqlens[n], cu_seqlens[n+1]); without it N = B and every
  * sequence has T tokens.
@@ -113,11 +119,13 @@ static void update_form3(double *S, const double *k, const double *v, double alp
 int oracle_run(const double *q, const double *k, const double *v, const double *g,
                const double *beta, const double *state_in, const int32_t *cu_seqlens,
                int n_seqs, int B, int T, int Hqk, int Hv, int dk, int dv, double scale,
-               int form, int n_threads, double *o, double *state_out) {
+               int form, int n_threads, double *o, double *state_out, int chunk_len,
+               double *chunk_states) {
   if (!q || !k || !v || !beta || !o) return ORACLE_EARG;
   if (B < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return ORACLE_EARG;
   if (Hv % Hqk != 0) return ORACLE_EARG;
   if (form < 1 || form > 3) return ORACLE_EARG;
+  if (chunk_states && chunk_len <= 0) return ORACLE_EARG;
   int N = cu_seqlens ? n_seqs : B;
   if (cu_seqlens) {
     if (B != 1 || n_seqs < 0) return ORACLE_EARG;
@@ -144,6 +152,13 @@ int oracle_run(const double *q, const double *k, const double *v, const double *
       b = n;
       t0 = 0;
       t1 = T;
+    }
+    long cbase = 0; /* first chunk_states row of sequence n */
+    if (chunk_states) {
+      for (int m = 0; m < n; ++m) {
+        const long len = cu_seqlens ? (long)cu_seqlens[m + 1] - cu_seqlens[m] : (long)T;
+        cbase += (len + chunk_len - 1) / chunk_len;
+      }
     }
     double *S = (double *)calloc((size_t)dv * dk, sizeof(double));
     double *A = form == 1 ? (double *)malloc(sizeof(double) * (size_t)dk * dk) : NULL;
@@ -180,6 +195,12 @@ int oracle_run(const double *q, const double *k, const double *v, const double *
         double acc = 0.0;
         for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * qs[i];
         ot[j] = acc;
+      }
+      if (chunk_states && ((t + 1 - t0) % chunk_len == 0 || t + 1 == t1)) {
+        const long row = cbase + (t - t0) / chunk_len;
+        double *Hc = chunk_states + ((size_t)row * Hv + h) * dk * dv;
+        for (int i = 0; i < dk; ++i)
+          for (int j = 0; j < dv; ++j) Hc[(size_t)i * dv + j] = S[(size_t)j * dk + i];
       }
     }
     if (state_out) {
