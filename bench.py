@@ -326,6 +326,37 @@ def run_ours(args, dist: Dist):
             "roofline": {"bound": "hbm", "frac": round(algo_bytes / (l_ms / 1e3) / 1e9 / hbm_peak, 4),
                          "peak": hbm_peak, "unit": "GB/s", "peak_kind": peak_kind},
         }
+        # the headline workload also returning the state after every 64-token chunk
+        n_cs = dr.chunk_state_rows(None, B, T)
+        cs = torch.empty((n_cs, Hv, dk, dv), dtype=torch.float32, device=dev)
+
+        def cs_step(_):
+            dr.chunk_fwd(p.q, p.k, p.v, p.g, p.beta, p.state_in, None, o=o, state_out=st,
+                         chunk_states=cs)
+
+        for i in range(2):
+            flush.zero_()
+            cs_step(i)
+        torch.cuda.synchronize()
+        assert dr.device_status(dev) == 0
+        dist.barrier()
+        c_durs = time_steps(cs_step, max(3, min(args.steps, 10)), stream, flush)
+        dist.barrier()
+        c_ms = dist.max(sum(c_durs) / len(c_durs), dev)
+        cs_bytes = algo_bytes + n_cs * Hv * dk * dv * 4
+        secondary["prefill_chunk_states"] = {
+            "metric": "prefill tokens/s also writing the state after every 64-token chunk "
+                      "(same workload)",
+            "value": round(dist.world * tokens / (c_ms / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(c_ms, 4), "chunk_state_bytes": n_cs * Hv * dk * dv * 4,
+            "roofline": {"bound": "hbm", "algorithmic_bytes_per_launch": cs_bytes,
+                         "achieved": round(cs_bytes / (c_ms / 1e3) / 1e9, 1),
+                         "frac": round(cs_bytes / (c_ms / 1e3) / 1e9 / hbm_peak, 4),
+                         "peak": hbm_peak, "unit": "GB/s", "peak_kind": peak_kind,
+                         "traffic": profiled_traffic(
+                             kfile, "gated_prefill_chunk_states_B2_T8192_Hqk16_Hv32_d128")},
+        }
+        del cs
         secondary["decode"] = bench_decode(dev, dist, stream, hbm_peak, peak_kind)
         secondary["varlen"] = bench_varlen(dev, dist, stream, flush, hbm_peak, peak_kind)
     clk = clocks.stop()

@@ -18,8 +18,8 @@ from typing import Optional
 
 import torch
 
-__all__ = ["chunk_fwd", "recurrent_step", "device_status", "prefill_kernel", "lib", "DrError",
-           "LIB_PATH"]
+__all__ = ["chunk_fwd", "recurrent_step", "device_status", "prefill_kernel", "chunk_state_rows",
+           "lib", "DrError", "LIB_PATH", "CHUNK"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdr.so")
 
@@ -48,7 +48,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         vp, fp, ip, i32 = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32
         L.dr_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i32, i32, i32, i32, i32, i32,
-                                   ctypes.c_int, ctypes.c_float, vp, ctypes.c_int, fp,
+                                   ctypes.c_int, ctypes.c_float, vp, ctypes.c_int, fp, fp,
                                    ctypes.c_uint32, vp]
         L.dr_chunk_fwd.restype = ctypes.c_int
         L.dr_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, i32,
@@ -94,9 +94,24 @@ def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+CHUNK = 64  # DR_CHUNK of include/dr.h: tokens between two returned chunk states
+
+
+def chunk_state_rows(cu_seqlens, B: int, T: int) -> int:
+    """Rows of the ``chunk_states`` output: ceil(max(len, 0) / CHUNK) per sequence.
+
+    ``cu_seqlens`` (a tensor or sequence, or None for B sequences of T tokens) is read on
+    the host; a device tensor is copied over (one synchronisation).
+    """
+    if cu_seqlens is None:
+        return B * (-(-T // CHUNK))
+    cu = cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else list(cu_seqlens)
+    return sum(-(-max(int(b) - int(a), 0) // CHUNK) for a, b in zip(cu[:-1], cu[1:]))
+
+
 def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
               output_final_state: bool = True, out_dtype=torch.float32, o=None, state_out=None,
-              qk_l2norm: bool = False):
+              qk_l2norm: bool = False, output_chunk_states: bool = False, chunk_states=None):
     """Chunked prefill through ``dr_chunk_fwd``.
 
     q, k [B, T, Hqk, dk] and v [B, T, Hv, dv] in bf16 or fp32 (same dtype);
@@ -104,6 +119,10 @@ def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1
     cu_seqlens int32 [N+1] (device) or None.  ``qk_l2norm``: the kernel divides every q and
     k row by its L2 norm first (``DR_QK_L2NORM``).  Returns (o [B, T, Hv, dv] in
     ``out_dtype``, state_out [N, Hv, dk, dv] fp32 or None).
+    ``output_chunk_states`` (or a given ``chunk_states`` tensor): a third output holds the
+    state after every ``CHUNK`` tokens of each sequence and after its last token,
+    [chunk_state_rows(cu_seqlens, B, T), Hv, dk, dv] fp32, sequence after sequence.
+    Allocating it with cu_seqlens reads cu_seqlens on the host.
     """
     if q.dtype not in _DTYPES or out_dtype not in _DTYPES:
         raise ValueError("q/k/v must be bf16 or fp32; out_dtype bf16 or fp32")
@@ -130,13 +149,22 @@ def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1
     if output_final_state and state_out is None:
         state_out = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=dev)
     _check(state_out, "state_out", torch.float32, dev)
+    want_cs = output_chunk_states or chunk_states is not None
+    if want_cs:
+        rows = chunk_state_rows(cu_seqlens, B, T)
+        if chunk_states is None:
+            chunk_states = torch.empty((rows, Hv, dk, dv), dtype=torch.float32, device=dev)
+        elif tuple(chunk_states.shape) != (rows, Hv, dk, dv):
+            raise ValueError(f"chunk_states must be {(rows, Hv, dk, dv)}")
+        _check(chunk_states, "chunk_states", torch.float32, dev)
     rc = lib().dr_chunk_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), N,
         B, T, Hqk, Hv, dk, dv, _DTYPES[q.dtype], float(scale), _ptr(o), _DTYPES[out_dtype],
-        _ptr(state_out), QK_L2NORM if qk_l2norm else 0, _stream(dev))
+        _ptr(state_out), _ptr(chunk_states) if want_cs else None,
+        QK_L2NORM if qk_l2norm else 0, _stream(dev))
     if rc != 0:
         raise DrError(rc, "dr_chunk_fwd")
-    return o, state_out
+    return (o, state_out, chunk_states) if want_cs else (o, state_out)
 
 
 def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.float32, o=None,

@@ -176,9 +176,12 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_
   lo = tc::pack_bf16(x0 - h0, x1 - h1);
 }
 
-// L2N: q and k rows are L2-normalised first (a compile-time switch, so that the plain path
-// carries none of its code).
-template <bool OUT_F32, bool L2N>
+static_assert(C == STATE_CHUNK, "one stored state per chunk");
+
+// L2N: q and k rows are L2-normalised first; CS: the state after every chunk is stored to
+// a.chunk_states.  Both are compile-time switches, so that the plain path carries none of
+// their code.
+template <bool OUT_F32, bool L2N, bool CS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     chunk_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -690,6 +693,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
     } else if (wg == 1 || wg == 2) {
       // ------------------------------------------------ state chain (fp32 state in registers)
       const int swg = wg - 1, st = tid - 128;  // swg: key rows [64 swg, +64), r columns [32 swg, +32)
+      long long cbase = 0;  // first chunk-state row of this sequence
+      if constexpr (CS) cbase = chunk_row_base(a.cu_seqlens, n, a.T, C);
       float Hr[64];
 #pragma unroll
       for (int m = 0; m < 64; ++m)
@@ -753,6 +758,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NT, 1)
         }
         tck::warp_arrive(bar(S_H0_FULL), lane);
         tck::warp_arrive(bar(S_GATE_EMPTY + s), lane);
+        if constexpr (CS) {
+          // after the arrivals: the stores leave the chain's critical path
+          float *hc = a.chunk_states + ((size_t)(cbase + c) * a.Hv + h) * DK * DV;
+#pragma unroll
+          for (int m = 0; m < 64; ++m) hc[(size_t)(64 * swg + m) * DV + row] = Hr[m];
+        }
       }
       if (a.state_out) {
 #pragma unroll
@@ -844,10 +855,14 @@ inline cudaError_t pair_dispatch(bool out_f32, const PrefillArgs &a, int N, cuda
       !tck::make_map(&mv, a.v, 128, a.Hv, rows) ||
       !tck::make_map_out(&mo, a.o, 128, a.Hv, rows, out_f32))
     return cudaErrorInvalidValue;
-  auto kern = out_f32 ? (a.qk_l2norm ? tcp::chunk_pair_kernel<true, true>
-                                     : tcp::chunk_pair_kernel<true, false>)
-                      : (a.qk_l2norm ? tcp::chunk_pair_kernel<false, true>
-                                     : tcp::chunk_pair_kernel<false, false>);
+  using Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                       const CUtensorMap, PrefillArgs);
+  static constexpr Kern kerns[8] = {
+      tcp::chunk_pair_kernel<false, false, false>, tcp::chunk_pair_kernel<false, false, true>,
+      tcp::chunk_pair_kernel<false, true, false>,  tcp::chunk_pair_kernel<false, true, true>,
+      tcp::chunk_pair_kernel<true, false, false>,  tcp::chunk_pair_kernel<true, false, true>,
+      tcp::chunk_pair_kernel<true, true, false>,   tcp::chunk_pair_kernel<true, true, true>};
+  const Kern kern = kerns[(out_f32 ? 4 : 0) + (a.qk_l2norm ? 2 : 0) + (a.chunk_states ? 1 : 0)];
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)tcp::SMEM_BYTES);
   if (e != cudaSuccess) return e;

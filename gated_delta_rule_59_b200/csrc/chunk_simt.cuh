@@ -34,7 +34,11 @@ struct PrefillArgs {
   void *o;
   float *state_out;
   int qk_l2norm;  // 1: divide q and k rows by their L2 norms first (zero rows stay zero)
+  float *chunk_states;  // [rows, Hv, dk, dv] state after every 64 tokens, or null
 };
+
+// Token count between two stored chunk states (the tensor-core kernel's chunk length).
+constexpr int STATE_CHUNK = DR_CHUNK;
 
 template <int DK, int DVS, int C>
 struct SimtSmem {
@@ -80,6 +84,9 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(PrefillArgs a, int dv) 
     const int i = idx / DVS, j = idx % DVS;
     Hs[i * VP + j] = a.state_in ? a.state_in[st_off + (size_t)i * dv + j0 + j] : 0.f;
   }
+
+  const long long cbase =
+      a.chunk_states ? chunk_row_base(a.cu_seqlens, n, a.T, STATE_CHUNK) : 0;
 
   for (int c0 = bos; c0 < eos; c0 += C) {
     const int L = min(C, eos - c0);
@@ -221,13 +228,19 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(PrefillArgs a, int dv) 
       io<Tout>::st(o + (((size_t)batch * a.T + c0 + r) * a.Hv + h) * dv + j0 + j, out);
     }
     __syncthreads();
-    // ---- H = gamma_last H0 + Ktil^T Delta ----
+    // ---- H = gamma_last H0 + Ktil^T Delta; stored too at a 64-token boundary ----
     const float glast = expf(blast);
+    const bool keep = a.chunk_states && ((c0 + L - bos) % STATE_CHUNK == 0 || c0 + L == eos);
+    float *hc = keep ? a.chunk_states +
+                           ((size_t)(cbase + (c0 - bos) / STATE_CHUNK) * a.Hv + h) * DK * dv + j0
+                     : nullptr;
     for (int idx = tid; idx < DK * DVS; idx += NT) {
       const int i = idx / DVS, j = idx % DVS;
       float acc = 0.f;
       for (int s = 0; s < C; ++s) acc += ktil[s] * Ks[s * KP + i] * Ds[s * VP + j];
-      Hs[i * VP + j] = glast * Hs[i * VP + j] + acc;
+      const float hn = glast * Hs[i * VP + j] + acc;
+      Hs[i * VP + j] = hn;
+      if (keep) hc[(size_t)i * dv + j] = hn;
     }
   }
   __syncthreads();
@@ -243,6 +256,7 @@ template <int DK, int DV, typename Tin, typename Tout>
 cudaError_t launch_chunk_simt(const PrefillArgs &a, int N, cudaStream_t stream) {
   constexpr int DVS = DV < 32 ? DV : 32;
   constexpr int C = 32;
+  static_assert(STATE_CHUNK % C == 0, "chunk states are taken at chunk ends");
   using SM = SimtSmem<DK, DVS, C>;
   auto kern = chunk_simt_kernel<DK, DVS, C, Tin, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -55,4 +55,20 @@ __device__ __forceinline__ bool seq_bounds(const int32_t *cu_seqlens, int n, int
   return true;
 }
 
+// First chunk-state row of sequence n: the number of 64-token chunks (a ragged last one
+// included) of the sequences before it, a sequence of length <= 0 counting none.  Without
+// cu_seqlens every sequence has T tokens.  Called by a whole, converged warp.
+__device__ __forceinline__ long long chunk_row_base(const int32_t *cu_seqlens, int n, int T,
+                                                    int chunk) {
+  if (cu_seqlens == nullptr) return (long long)n * ((T + chunk - 1) / chunk);
+  long long rows = 0;
+  for (int m = (int)(threadIdx.x & 31); m < n; m += 32) {
+    const long long len = (long long)cu_seqlens[m + 1] - cu_seqlens[m];
+    rows += len > 0 ? (len + chunk - 1) / chunk : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rows += __shfl_xor_sync(0xffffffffu, rows, o);
+  return rows;
+}
+
 }  // namespace dr

@@ -63,7 +63,8 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
                        const float *beta, const float *state_in, const int32_t *cu_seqlens,
                        int32_t n_seqs, int32_t B, int32_t T, int32_t Hqk, int32_t Hv,
                        int32_t dk, int32_t dv, dr_dtype in_dtype, float scale, void *o,
-                       dr_dtype o_dtype, float *state_out, uint32_t flags, dr_stream stream) {
+                       dr_dtype o_dtype, float *state_out, float *chunk_states,
+                       uint32_t flags, dr_stream stream) {
   if (!dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return DR_ERR_DTYPE;
   if (flags & ~DR_QK_L2NORM) return DR_ERR_UNSUPPORTED;
   if (B < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return DR_ERR_SHAPE;
@@ -75,7 +76,8 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
   const bool tokens = (int64_t)B * T > 0;
   if (tokens && (!q || !k || !v || !beta || !o)) return DR_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-      !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(g, 4) ||
+      !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(chunk_states, 16) ||
+      !aligned(g, 4) ||
       !aligned(beta, 4) || !aligned(cu_seqlens, 4))
     return DR_ERR_ALIGN;
   if (N == 0) return DR_OK;
@@ -83,7 +85,7 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   dr::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, (int)N, B, T, Hqk, Hv,
-                    scale, o, state_out, (flags & DR_QK_L2NORM) ? 1 : 0};
+                    scale, o, state_out, (flags & DR_QK_L2NORM) ? 1 : 0, chunk_states};
   cudaError_t e;
   if (in_dtype == DR_BF16 && dr::tc_supported(dk, dv)) {
     e = dr::prefill_tc_dispatch(dk, dv, o_dtype == DR_F32, a, (int)N, s);

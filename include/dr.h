@@ -63,6 +63,9 @@ typedef enum { DR_F32 = 0, DR_BF16 = 1 } dr_dtype;
 /* Same type as cudaStream_t. */
 typedef struct CUstream_st *dr_stream;
 
+/* Tokens per chunk of dr_chunk_fwd: the spacing of the states it returns in chunk_states. */
+#define DR_CHUNK 64
+
 /* Option bits of dr_chunk_fwd / dr_recurrent_step (any other bit => DR_ERR_UNSUPPORTED). */
 #define DR_QK_L2NORM 1u /* divide every q and k row (per token and q/k head) by its L2 norm
                            first (an all-zero row stays zero): the pages' qk_l2norm step
@@ -89,6 +92,15 @@ typedef struct CUstream_st *dr_stream;
  *   o          [B, T, Hv, dv]    o_dtype (DR_F32 or DR_BF16); every token's output is written
  *   state_out  [N, Hv, dk, dv] f32 or NULL (=> final state not returned).  It may be
  *              state_in itself (in-place update); a partial overlap is undefined.
+ *   chunk_states [R, Hv, dk, dv] f32 or NULL (=> not returned): the intermediate states
+ *              the "linear_attention" page's recurrent route exposes, sampled at chunk ends: the
+ *              state after every DR_CHUNK tokens of each sequence and after its last
+ *              token.  Sequence n owns ceil(max(len_n, 0) / DR_CHUNK) rows, in sequence
+ *              order, so R = sum_n of that count (N * ceil(T / DR_CHUNK) without
+ *              cu_seqlens); row j of a sequence holds the state after
+ *              min((j + 1) DR_CHUNK, len_n) tokens, and its last row equals its
+ *              state_out.  Caller-owned, 16-byte aligned, overlapping no other
+ *              argument; rows of a sequence that a bad cu_seqlens skips are not written.
  *   flags      0 or DR_QK_L2NORM
  *   T = 0 or N = 0 is valid: nothing is read from q/k/v; state_out (if given) receives
  *   state_in (or zeros).
@@ -98,7 +110,8 @@ DR_API dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const
                               const int32_t *cu_seqlens, int32_t n_seqs, int32_t B, int32_t T,
                               int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv,
                               dr_dtype in_dtype, float scale, void *o, dr_dtype o_dtype,
-                              float *state_out, uint32_t flags, dr_stream stream);
+                              float *state_out, float *chunk_states, uint32_t flags,
+                              dr_stream stream);
 
 /* Which prefill kernel dr_chunk_fwd launches for these inputs (host only, no device call). */
 typedef enum {

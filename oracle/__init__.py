@@ -123,8 +123,8 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
     With ``chunk_len`` > 0 a third array is returned: the stored state after every
     ``chunk_len`` tokens of each sequence and after its last token,
     [sum_n ceil(len_n / chunk_len), Hv, dk, dv], rows ordered as ``chunk_rows`` gives.
-    This is the intermediate state the "DeltaNet" tracing route exposes (the state after
-    every token, of which these are the chunk-boundary samples).
+    These sample, at chunk boundaries, the state after every token that the
+    "linear_attention" page (LinearAttention, its recurrent route) exposes for tracing.
     """
     lib = _load()
     q, k, v, g, beta, state_in = (_f64(a) for a in (q, k, v, g, beta, state_in))

@@ -55,9 +55,10 @@ P4 = ctypes.c_void_p(0x10004)
 
 
 def chunk(L, q=P16, k=P16, v=P16, g=None, beta=P16, s_in=None, cu=None, n_seqs=0, B=1, T=8,
-          Hqk=1, Hv=1, dk=64, dv=64, dt=1, scale=1.0, o=P16, odt=0, s_out=None, flags=0):
+          Hqk=1, Hv=1, dk=64, dv=64, dt=1, scale=1.0, o=P16, odt=0, s_out=None, cs=None,
+          flags=0):
     return L.dr_chunk_fwd(q, k, v, g, beta, s_in, cu, n_seqs, B, T, Hqk, Hv, dk, dv, dt, scale,
-                          o, odt, s_out, flags, None)
+                          o, odt, s_out, cs, flags, None)
 
 
 def step(L, q=P16, k=P16, v=P16, g=None, beta=P16, state=P16, B=2, Hqk=1, Hv=1, dk=64, dv=64,
@@ -83,6 +84,8 @@ def test_chunk_fwd_argument_errors(L):
     assert chunk(L, q=ctypes.c_void_p(0x10008)) == 4
     assert chunk(L, s_in=ctypes.c_void_p(0x10004)) == 4
     assert chunk(L, g=ctypes.c_void_p(0x10002)) == 4
+    assert chunk(L, cs=ctypes.c_void_p(0x10008)) == 4
+    assert chunk(L, cs=P16, B=0) == 0
     # option bits: DR_QK_L2NORM (1) is known, any other bit is unsupported
     assert chunk(L, flags=2) == 5
     assert chunk(L, flags=0x80000001) == 5
@@ -106,6 +109,19 @@ def test_recurrent_step_argument_errors(L):
     assert step(L, flags=4) == 5
     assert step(L, B=0, flags=1) == 0
     assert step(L, B=0) == 0
+
+
+def test_chunk_state_rows():
+    assert dr.CHUNK == 64
+    assert int(re.search(r"#define DR_CHUNK (\d+)", open(HEADER).read()).group(1)) == dr.CHUNK
+    assert dr.chunk_state_rows(None, 3, 130) == 9
+    assert dr.chunk_state_rows(None, 2, 0) == 0
+    assert dr.chunk_state_rows([0, 64, 64, 65, 200], 1, 200) == 1 + 0 + 1 + 3
+    # a decreasing (malformed) step counts no rows, as the kernels count it
+    assert dr.chunk_state_rows([0, 100, 50, 200], 1, 200) == 2 + 0 + 3
+    import oracle
+    for cu in ([0, 5, 5, 12], [0, 64, 129, 129, 300]):
+        assert dr.chunk_state_rows(cu, 1, cu[-1]) == oracle.chunk_rows(cu, 1, cu[-1], 64)[1]
 
 
 def test_binding_rejects_cpu_tensors():

@@ -1,8 +1,9 @@
 """Pins of the oracle's chunk-state output (the state at every chunk boundary).
 
-The "DeltaNet" page's tracing route exposes the state after every token; the oracle
-samples it after every ``chunk_len`` tokens of each sequence and after the sequence's
-last token.  Checked against things other than the token loop that writes them:
+The "linear_attention" page's recurrent route (LinearAttention) exposes the state
+after every token; the oracle samples it after every ``chunk_len`` tokens of each
+sequence and after the sequence's last token.  Checked against things other than the
+token loop that writes them:
   CS1  exact rational brute force on every prefix (closed product of affine maps),
        varlen with an empty sequence and a ragged tail, dk != dv;
   CS2  the chunk (UT/WY) form's own end-of-chunk states, for several chunk lengths;
