@@ -55,7 +55,7 @@ def _load():
             dp, dp, dp, dp, dp, dp, ip,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int,
-            dp, dp, ctypes.c_int, dp,
+            dp, dp, ctypes.c_int, dp, ctypes.c_int,
         ]
         lib.oracle_run.restype = ctypes.c_int
         lib.oracle_max_threads.restype = ctypes.c_int
@@ -117,6 +117,8 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
     """Token-by-token fp64 recurrence.
 
     q, k: [B, T, Hqk, dk]; v: [B, T, Hv, dv]; g, beta: [B, T, Hv] (g may be None);
+    g may also be [B, T, Hv, dk]: one log decay per key channel (the "linear_attention"
+    page's ChannelGates), which scales row i of the stored state by exp(g[..., i]);
     state_in: [N, Hv, dk, dv] or None (zeros); cu_seqlens: int [N+1] or None.
     ``qk_l2norm``: q and k rows are L2-normalised first (``l2_normalize_rows``).
     Returns (o [B, T, Hv, dv], state_out [N, Hv, dk, dv]) as float64 numpy arrays.
@@ -133,8 +135,9 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
     B, T, Hqk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     assert k.shape == q.shape and v.shape[:2] == (B, T) and beta.shape == (B, T, Hv)
+    channel_gates = g is not None and g.ndim == 4
     if g is not None:
-        assert g.shape == (B, T, Hv)
+        assert g.shape == ((B, T, Hv, dk) if channel_gates else (B, T, Hv)), g.shape
     cu = None
     if cu_seqlens is not None:
         if hasattr(cu_seqlens, "detach"):
@@ -153,7 +156,7 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1.0,
     rc = lib.oracle_run(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
         _ptr(cu, ctypes.c_int32), N, B, T, Hqk, Hv, dk, dv, float(scale), int(form),
-        int(threads), _ptr(o), _ptr(st), int(chunk_len), _ptr(cs),
+        int(threads), _ptr(o), _ptr(st), int(chunk_len), _ptr(cs), int(channel_gates),
     )
     if rc != 0:
         raise ValueError(f"oracle_run failed with code {rc}")
@@ -164,7 +167,8 @@ def step(q, k, v, g, beta, state, scale: float = 1.0, form: int = 2, threads: in
          qk_l2norm: bool = False):
     """One decode step (T = 1) for every (batch, v-head).
 
-    q, k: [B, Hqk, dk]; v: [B, Hv, dv]; g, beta: [B, Hv]; state: [B, Hv, dk, dv].
+    q, k: [B, Hqk, dk]; v: [B, Hv, dv]; g, beta: [B, Hv] (g may be [B, Hv, dk]: per key
+    channel); state: [B, Hv, dk, dv].
     Returns (o [B, Hv, dv], new_state [B, Hv, dk, dv]); ``state`` is not modified.
     """
     q, k, v, beta, state = (_f64(a) for a in (q, k, v, beta, state))

@@ -12,7 +12,9 @@ A_t = alpha_t (I - beta_t k_t k_t^T), its solution is the closed product
 
 evaluated here with ``fractions.Fraction`` (no rounding at all) by forming the
 products explicitly, never by stepping the recurrence.  alpha_t is supplied
-directly as a rational number (exp(g) is not rational).
+directly as a rational number (exp(g) is not rational).  With per-key-channel
+gates (the "linear_attention" page's ChannelGates) alpha_t is a vector and
+A_t = diag(alpha_t) (I - beta_t k_t k_t^T).
 """
 from __future__ import annotations
 
@@ -32,6 +34,8 @@ def _eye(n):
 def solve(q, k, v, alpha, beta, S0):
     """q, k: T x dk; v: T x dv; alpha, beta: T; S0: dv x dk (all Fractions).
 
+    alpha[t] may be a list of dk Fractions (one decay per key channel).
+
     Returns (o: T x dv, S_T: dv x dk), exact.
     """
     T = len(k)
@@ -39,7 +43,8 @@ def solve(q, k, v, alpha, beta, S0):
     dv = len(v[0])
     A = []
     for t in range(T):
-        At = [[alpha[t] * ((1 if a == b else 0) - beta[t] * k[t][a] * k[t][b]) for b in range(dk)]
+        al = alpha[t] if isinstance(alpha[t], (list, tuple)) else [alpha[t]] * dk
+        At = [[al[a] * ((1 if a == b else 0) - beta[t] * k[t][a] * k[t][b]) for b in range(dk)]
               for a in range(dk)]
         A.append(At)
 

@@ -47,6 +47,35 @@ def chunk_step(Q, K, V, g, beta, H0):
     return O, H1
 
 
+def chunk_step_channel(Q, K, V, g, beta, H0):
+    """One chunk with per-key-channel gates g [L, dk] (the "linear_attention" page's
+    ChannelGates).  Same returns as ``chunk_step``.
+
+    With b_r = sum_{i<=r} g_i now a vector, the decay between tokens s <= r is
+    diag(exp(b_r - b_s)) and no longer factors out of the key products:
+        A_rs = sum_c k_r[c] k_s[c] exp(b_r[c] - b_s[c]),   Lmat = strict_lower(diag(beta) A)
+        W = T diag(beta) (K o e^b),   U = T diag(beta) V,   Delta = U - W H0
+        P_rs = sum_c q_r[c] k_s[c] exp(b_r[c] - b_s[c]) (s <= r)
+        O = (Q o e^b) H0 + P Delta,   H_L = diag(e^{b_{L-1}}) H0 + (K o e^{b_{L-1} - b})^T Delta
+    (o: elementwise, rows broadcast).  The scalar form is the case of equal columns.
+    """
+    L = K.shape[0]
+    b = np.cumsum(g, axis=0)                              # [L, dk]
+    incl = np.tril(np.ones((L, L), dtype=bool))
+    diff = b[:, None, :] - b[None, :, :]                  # [L, L, dk], r - s
+    E = np.where(incl[:, :, None], np.exp(np.where(incl[:, :, None], diff, 0.0)), 0.0)
+    A = np.einsum("rc,sc,rsc->rs", K, K, E)
+    Lmat = np.tril(beta[:, None] * A, k=-1)
+    T = np.linalg.inv(np.eye(L) + Lmat)
+    W = T @ (beta[:, None] * (K * np.exp(b)))
+    U = T @ (beta[:, None] * V)
+    Delta = U - W @ H0
+    P = np.einsum("rc,sc,rsc->rs", Q, K, E)
+    O = (Q * np.exp(b)) @ H0 + P @ Delta
+    H1 = np.exp(b[-1])[:, None] * H0 + (K * np.exp(b[-1] - b)).T @ Delta
+    return O, H1
+
+
 def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale=1.0, chunk=64,
         chunk_states=False):
     """Chunk form over a whole (possibly varlen-packed) batch.
@@ -60,6 +89,7 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale=1.0, chunk=64,
     B, T, Hqk, dk = q.shape
     Hv, dv = v.shape[2], v.shape[3]
     g = np.zeros((B, T, Hv)) if g is None else np.asarray(g, dtype=np.float64)
+    step = chunk_step_channel if g.ndim == 4 else chunk_step
     if cu_seqlens is not None:
         cu = [int(x) for x in np.asarray(cu_seqlens)]
         seqs = [(0, cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
@@ -77,8 +107,8 @@ def run(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale=1.0, chunk=64,
             H = np.zeros((dk, dv)) if state_in is None else np.array(state_in[n, h], dtype=np.float64)
             for c0 in range(t0, t1, chunk):
                 c1 = min(c0 + chunk, t1)
-                O, H = chunk_step(scale * q[bb, c0:c1, hq], k[bb, c0:c1, hq], v[bb, c0:c1, h],
-                                  g[bb, c0:c1, h], beta[bb, c0:c1, h], H)
+                O, H = step(scale * q[bb, c0:c1, hq], k[bb, c0:c1, hq], v[bb, c0:c1, h],
+                            g[bb, c0:c1, h], beta[bb, c0:c1, h], H)
                 o[bb, c0:c1, h] = O
                 cs[rows.index((n, c0)), h] = H
             st[n, h] = H

@@ -36,6 +36,12 @@
  *   form 3  retrieve-and-replace: v_old = S' k, v_new = beta v + (1-beta) v_old,
  *           S = S' - v_old k^T + v_new k^T.
  *
+ * Per-key-channel gates (channel_gates = 1): the "linear_attention" page's
+ * ChannelGates, [batch, seq, heads, key_dim], the gate of the KDA subclass.
+ * Read as one log kept-fraction per key channel: S' = S diag(alpha_t), i.e.
+ * column i of S (row i of the stored state) decays by exp(g_t[i]); the delta
+ * write that follows is unchanged.  A scalar gate is the case of equal entries.
+ *
  * Readings where the pages are silent: the decay multiplies the state before
  * the delta write; the query reads after the write; `scale` multiplies q
  * (1.0 reproduces o = S q); query/key head h_qk = h_v / (Hv / Hqk).
@@ -102,7 +108,8 @@ static void update_form3(double *S, const double *k, const double *v, double alp
  * Layouts (all host, contiguous, row-major, double):
  *   q, k        [B, T, Hqk, dk]
  *   v, o        [B, T, Hv, dv]
- *   g, beta     [B, T, Hv]        (g may be NULL: no decay)
+ *   g, beta     [B, T, Hv]        (g may be NULL: no decay); with channel_gates
+ *               g is [B, T, Hv, dk], one log decay per key channel
  *   state_in    [N, Hv, dk, dv]   (may be NULL: zero state)
  *   state_out   [N, Hv, dk, dv]   (may be NULL)
  *   chunk_states [NC, Hv, dk, dv] (may be NULL): the stored state S^T after
@@ -120,7 +127,7 @@ int oracle_run(const double *q, const double *k, const double *v, const double *
                const double *beta, const double *state_in, const int32_t *cu_seqlens,
                int n_seqs, int B, int T, int Hqk, int Hv, int dk, int dv, double scale,
                int form, int n_threads, double *o, double *state_out, int chunk_len,
-               double *chunk_states) {
+               double *chunk_states, int channel_gates) {
   if (!q || !k || !v || !beta || !o) return ORACLE_EARG;
   if (B < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return ORACLE_EARG;
   if (Hv % Hqk != 0) return ORACLE_EARG;
@@ -180,9 +187,16 @@ int oracle_run(const double *q, const double *k, const double *v, const double *
       const double *kt = k + (tok * Hqk + hq) * dk;
       const double *qt = q + (tok * Hqk + hq) * dk;
       const double *vt = v + (tok * Hv + h) * dv;
-      const double gt = g ? g[tok * Hv + h] : 0.0;
       const double bt = beta[tok * Hv + h];
-      const double alpha = exp(gt);
+      double alpha = 1.0;
+      if (g && channel_gates) {
+        /* S' = S diag(alpha_t): column i of S scales by exp(g_t[i]) */
+        const double *gt = g + (tok * Hv + h) * dk;
+        for (int j = 0; j < dv; ++j)
+          for (int i = 0; i < dk; ++i) S[(size_t)j * dk + i] *= exp(gt[i]);
+      } else if (g) {
+        alpha = exp(g[tok * Hv + h]);
+      }
       if (form == 1)
         update_form1(S, A, kt, vt, alpha, bt, dk, dv);
       else if (form == 2)
