@@ -357,6 +357,8 @@ def run_ours(args, dist: Dist):
                              kfile, "gated_prefill_chunk_states_B2_T8192_Hqk16_Hv32_d128")},
         }
         del cs
+        secondary["prefill_channel_gates"] = bench_channel_gates(dev, dist, stream, flush,
+                                                                hbm_peak, peak_kind, args)
         secondary["decode"] = bench_decode(dev, dist, stream, hbm_peak, peak_kind)
         secondary["varlen"] = bench_varlen(dev, dist, stream, flush, hbm_peak, peak_kind)
     clk = clocks.stop()
@@ -380,6 +382,40 @@ def run_ours(args, dist: Dist):
     dist.close()
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def bench_channel_gates(dev, dist, stream, flush, hbm_peak, peak_kind, args):
+    """The headline shape with per-key-channel gates (g [B, T, Hv, dk]): the CUDA-core kernel."""
+    import gated_delta_rule_59_b200 as dr
+    from gated_delta_rule_59_b200 import inputs
+
+    B, T, Hqk, Hv, d = 2, 8192, 16, 32, 128
+    p = inputs.prefill(B, T, Hqk, Hv, d, d, torch.bfloat16, gated=True, state_std=0.02,
+                       seed=inputs.SEED_BASE + 2, channel_gates=True).to(dev)
+    o = torch.empty((B, T, Hv, d), dtype=torch.float32, device=dev)
+    st = torch.empty((B, Hv, d, d), dtype=torch.float32, device=dev)
+
+    def step(_):
+        dr.chunk_fwd(p.q, p.k, p.v, p.g, p.beta, p.state_in, None, o=o, state_out=st)
+
+    for i in range(2):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    assert dr.device_status(dev) == 0
+    dist.barrier()
+    durs = time_steps(step, 3, stream, flush)
+    dist.barrier()
+    ms = dist.max(sum(durs) / len(durs), dev)
+    algo = prefill_bytes(B, T, Hqk, Hv, d, d, 2, 4, B, True) + B * T * Hv * (d - 1) * 4
+    return {
+        "metric": "prefill tokens/s with per-key-channel gates (same shape; CUDA-core kernel)",
+        "value": round(dist.world * B * T / (ms / 1e3), 1), "unit": "tokens/s",
+        "ms_per_step": round(ms, 4), "kernel": dr.prefill_kernel(torch.bfloat16, d, d, True),
+        "roofline": {"bound": "alu", "hbm_frac": round(algo / (ms / 1e3) / 1e9 / hbm_peak, 4),
+                     "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind},
+        "gpu_launches": 3,
+    }
 
 
 def bench_decode(dev, dist, stream, hbm_peak, peak_kind):

@@ -116,6 +116,8 @@ def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1
 
     q, k [B, T, Hqk, dk] and v [B, T, Hv, dv] in bf16 or fp32 (same dtype);
     g (or None), beta [B, T, Hv] fp32; state_in [N, Hv, dk, dv] fp32 or None;
+    g may be [B, T, Hv, dk] instead: one log decay per key channel (``DR_GATE_PER_CHANNEL``,
+    the "linear_attention" page's ChannelGates), run by the CUDA-core kernel.
     cu_seqlens int32 [N+1] (device) or None.  ``qk_l2norm``: the kernel divides every q and
     k row by its L2 norm first (``DR_QK_L2NORM``).  Returns (o [B, T, Hv, dv] in
     ``out_dtype``, state_out [N, Hv, dk, dv] fp32 or None).
@@ -138,8 +140,9 @@ def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1
     Hv, dv = v.shape[2], v.shape[3]
     if k.shape != q.shape or v.shape[:2] != (B, T) or beta.shape != (B, T, Hv):
         raise ValueError("inconsistent shapes")
-    if g is not None and g.shape != (B, T, Hv):
-        raise ValueError("g must be [B, T, Hv]")
+    channel_gates = g is not None and g.dim() == 4
+    if g is not None and tuple(g.shape) not in ((B, T, Hv), (B, T, Hv, dk)):
+        raise ValueError("g must be [B, T, Hv] or [B, T, Hv, dk]")
     N = B if cu_seqlens is None else cu_seqlens.numel() - 1
     if state_in is not None and tuple(state_in.shape) != (N, Hv, dk, dv):
         raise ValueError(f"state_in must be {(N, Hv, dk, dv)}")
@@ -161,7 +164,8 @@ def chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None, scale: float = 1
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in), _ptr(cu_seqlens), N,
         B, T, Hqk, Hv, dk, dv, _DTYPES[q.dtype], float(scale), _ptr(o), _DTYPES[out_dtype],
         _ptr(state_out), _ptr(chunk_states) if want_cs else None,
-        QK_L2NORM if qk_l2norm else 0, _stream(dev))
+        (QK_L2NORM if qk_l2norm else 0) | (GATE_PER_CHANNEL if channel_gates else 0),
+        _stream(dev))
     if rc != 0:
         raise DrError(rc, "dr_chunk_fwd")
     return (o, state_out, chunk_states) if want_cs else (o, state_out)
@@ -172,7 +176,7 @@ def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.
     """One decode step through ``dr_recurrent_step``; ``state`` is updated in place.
 
     q, k [B, Hqk, dk], v [B, Hv, dv] (bf16 or fp32); g (or None), beta [B, Hv] fp32;
-    state [B, Hv, dk, dv] fp32.  ``qk_l2norm`` as for ``chunk_fwd``.  Returns o [B, Hv, dv] in
+    g may be [B, Hv, dk] (per key channel, as for ``chunk_fwd``); state [B, Hv, dk, dv] fp32.  ``qk_l2norm`` as for ``chunk_fwd``.  Returns o [B, Hv, dv] in
     ``out_dtype``.
     """
     if q.dtype not in _DTYPES or out_dtype not in _DTYPES:
@@ -186,13 +190,17 @@ def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.
     Hv, dv = v.shape[1], v.shape[2]
     if tuple(state.shape) != (B, Hv, dk, dv) or beta.shape != (B, Hv):
         raise ValueError("inconsistent shapes")
+    channel_gates = g is not None and g.dim() == 3
+    if g is not None and tuple(g.shape) not in ((B, Hv), (B, Hv, dk)):
+        raise ValueError("g must be [B, Hv] or [B, Hv, dk]")
     if o is None:
         o = torch.empty((B, Hv, dv), dtype=out_dtype, device=dev)
     _check(o, "o", out_dtype, dev)
     rc = lib().dr_recurrent_step(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), B, Hqk, Hv, dk, dv,
         _DTYPES[q.dtype], float(scale), _ptr(o), _DTYPES[out_dtype],
-        QK_L2NORM if qk_l2norm else 0, _stream(dev))
+        (QK_L2NORM if qk_l2norm else 0) | (GATE_PER_CHANNEL if channel_gates else 0),
+        _stream(dev))
     if rc != 0:
         raise DrError(rc, "dr_recurrent_step")
     return o
@@ -200,11 +208,13 @@ def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.
 
 KERNELS = {0: None, 1: "simt_f32", 2: "tc_bf16"}
 QK_L2NORM = 1  # DR_QK_L2NORM of include/dr.h
+GATE_PER_CHANNEL = 2  # DR_GATE_PER_CHANNEL of include/dr.h
 
 
-def prefill_kernel(dtype, dk: int, dv: int):
+def prefill_kernel(dtype, dk: int, dv: int, channel_gates: bool = False):
     """Name of the kernel dr_chunk_fwd picks for these inputs ('tc_bf16', 'simt_f32' or None)."""
-    return KERNELS[lib().dr_chunk_fwd_kernel(_DTYPES[dtype], dk, dv)]
+    name = KERNELS[lib().dr_chunk_fwd_kernel(_DTYPES[dtype], dk, dv)]
+    return "simt_f32" if (channel_gates and name is not None) else name
 
 
 def device_status(device=None) -> int:

@@ -16,6 +16,14 @@
 // Rows past the end of a sequence are padded with q = k = v = 0, beta = 0,
 // g = 0, which leaves Delta = 0 for them and changes nothing else.
 //
+// Per-key-channel gates (the "linear_attention" page's ChannelGates, g [.., dk]):
+// b_r is a vector and the decay between tokens s <= r, diag(e^{b_r - b_s}), no
+// longer factors out of the key products, so it goes inside them:
+//     A_rs = sum_i k_r[i] k_s[i] e^{b_r[i] - b_s[i]},  P_rs likewise with q_r;
+//     W = T diag(beta) (K o e^b),  O = (Q o e^b) H0 + P Delta,
+//     H = diag(e^{b_last}) H0 + (K o e^{b_last - b})^T Delta.
+// Every exponent is <= 0 for non-positive gates.
+//
 // One CTA owns one (sequence, v-head, dv-slice of DVS columns): the state
 // columns evolve independently given k, beta and g, so slices need no
 // communication; K K^T, Q K^T and T are recomputed per slice.
@@ -35,6 +43,7 @@ struct PrefillArgs {
   float *state_out;
   int qk_l2norm;  // 1: divide q and k rows by their L2 norms first (zero rows stay zero)
   float *chunk_states;  // [rows, Hv, dk, dv] state after every 64 tokens, or null
+  int channel_gates;    // 1: g is [B, T, Hv, dk], one log decay per key channel
 };
 
 // Token count between two stored chunk states (the tensor-core kernel's chunk length).
@@ -48,6 +57,8 @@ struct SimtSmem {
   static constexpr int floats =
       3 * C * KP + DK * VP + 3 * C * VP + 2 * C * CP + 4 * C;
   static constexpr size_t bytes = sizeof(float) * floats;
+  // per-key-channel gates add the cumulative decays b[r][i] and K o e^b
+  static constexpr size_t bytes_cg = bytes + sizeof(float) * 2 * C * KP;
 };
 
 template <int DK, int DVS, int C, typename Tin, typename Tout>
@@ -68,6 +79,9 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(PrefillArgs a, int dv) 
   float *betas = bs + C;        // [C]
   float *bgs = betas + C;       // [C] beta * gamma
   float *ktil = bgs + C;        // [C] e^{b_last - b_s}
+  float *Gb = ktil + C;         // [C][KP] channel gates: cumulative log decay b[r][i]
+  float *Kb = Gb + C * KP;      // [C][KP] channel gates: K o e^{b}
+  const bool cg = a.channel_gates != 0;
 
   const int tid = threadIdx.x;
   const int unit = blockIdx.x, n = unit / a.Hv, h = unit % a.Hv;
@@ -126,14 +140,31 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(PrefillArgs a, int dv) 
         }
       }
     }
+    if (cg) {
+      // per-key-channel gates: b[r][i] = sum of g over the chunk's rows <= r, per channel
+      for (int idx = tid; idx < C * DK; idx += NT) {
+        const int r = idx / DK, i = idx % DK;
+        Gb[r * KP + i] =
+            r < L ? a.g[(((size_t)batch * a.T + c0 + r) * a.Hv + h) * DK + i] : 0.f;
+      }
+      __syncthreads();
+      for (int i = tid; i < DK; i += NT) {
+        float acc = 0.f;
+        for (int r = 0; r < C; ++r) {
+          acc += Gb[r * KP + i];
+          Gb[r * KP + i] = acc;
+        }
+      }
+    }
     if (tid < 32) {
-      // inclusive prefix sum of g over the chunk (C <= 32 handled per lane)
+      // inclusive prefix sum of g over the chunk (C <= 32 handled per lane); with channel
+      // gates the scalar decay is 1 and b lives in Gb
       for (int base = 0; base < C; base += 32) {
         const int r = base + tid;
         float gv = 0.f, bv = 0.f;
         if (r < L) {
           const size_t go = ((size_t)batch * a.T + c0 + r) * a.Hv + h;
-          gv = a.g ? a.g[go] : 0.f;
+          gv = (a.g && !cg) ? a.g[go] : 0.f;
           bv = a.beta[go];
         }
 #pragma unroll
@@ -161,10 +192,18 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(PrefillArgs a, int dv) 
       float lv = 0.f, pv = 0.f;
       if (s <= r) {
         float akk = 0.f, aqk = 0.f;
-        for (int i = 0; i < DK; ++i) {
-          const float ks_ = Ks[s * KP + i];
-          akk += Ks[r * KP + i] * ks_;
-          aqk += Qs[r * KP + i] * ks_;
+        if (cg) {  // the decay between s and r differs per channel: inside the sums
+          for (int i = 0; i < DK; ++i) {
+            const float ks_ = Ks[s * KP + i] * expf(Gb[r * KP + i] - Gb[s * KP + i]);
+            akk += Ks[r * KP + i] * ks_;
+            aqk += Qs[r * KP + i] * ks_;
+          }
+        } else {
+          for (int i = 0; i < DK; ++i) {
+            const float ks_ = Ks[s * KP + i];
+            akk += Ks[r * KP + i] * ks_;
+            aqk += Qs[r * KP + i] * ks_;
+          }
         }
         const float gam = expf(bs[r] - bs[s]);
         pv = gam * aqk;
@@ -193,12 +232,25 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(PrefillArgs a, int dv) 
       for (int r = 0; r < C; ++r) Ls[r * CP + c] = col[r];
     }
     __syncthreads();
+    if (cg) {
+      // K -> K o e^{b} (into Kb, for W), K -> K o e^{b_last - b} (in place, for the state),
+      // Q -> Q o e^{b} (in place, for the read of H0)
+      for (int idx = tid; idx < C * DK; idx += NT) {
+        const int r = idx / DK, i = idx % DK;
+        const float b = Gb[r * KP + i], kv = Ks[r * KP + i];
+        Kb[r * KP + i] = kv * expf(b);
+        Ks[r * KP + i] = kv * expf(Gb[(C - 1) * KP + i] - b);
+        Qs[r * KP + i] *= expf(b);
+      }
+      __syncthreads();
+    }
     float *Ts = Ls;
+    const float *Kw = cg ? Kb : Ks;
     // ---- W = T diag(beta gamma) K, U = T diag(beta) V ----
     for (int idx = tid; idx < C * DK; idx += NT) {
       const int r = idx / DK, i = idx % DK;
       float acc = 0.f;
-      for (int s = 0; s <= r; ++s) acc += Ts[r * CP + s] * bgs[s] * Ks[s * KP + i];
+      for (int s = 0; s <= r; ++s) acc += Ts[r * CP + s] * bgs[s] * Kw[s * KP + i];
       Ws[r * KP + i] = acc;
     }
     for (int idx = tid; idx < C * DVS; idx += NT) {
@@ -238,7 +290,8 @@ __global__ void __launch_bounds__(256) chunk_simt_kernel(PrefillArgs a, int dv) 
       const int i = idx / DVS, j = idx % DVS;
       float acc = 0.f;
       for (int s = 0; s < C; ++s) acc += ktil[s] * Ks[s * KP + i] * Ds[s * VP + j];
-      const float hn = glast * Hs[i * VP + j] + acc;
+      const float gl = cg ? expf(Gb[(C - 1) * KP + i]) : glast;
+      const float hn = gl * Hs[i * VP + j] + acc;
       Hs[i * VP + j] = hn;
       if (keep) hc[(size_t)i * dv + j] = hn;
     }
@@ -259,11 +312,12 @@ cudaError_t launch_chunk_simt(const PrefillArgs &a, int N, cudaStream_t stream) 
   static_assert(STATE_CHUNK % C == 0, "chunk states are taken at chunk ends");
   using SM = SimtSmem<DK, DVS, C>;
   auto kern = chunk_simt_kernel<DK, DVS, C, Tin, Tout>;
+  const size_t smem = a.channel_gates ? SM::bytes_cg : SM::bytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SM::bytes);
+                                       (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)N * (unsigned)a.Hv, DV / DVS);
-  kern<<<grid, 256, SM::bytes, stream>>>(a, DV);
+  kern<<<grid, 256, smem, stream>>>(a, DV);
   return cudaGetLastError();
 }
 

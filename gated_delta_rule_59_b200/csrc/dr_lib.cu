@@ -25,11 +25,11 @@ bool dtype_ok(dr_dtype t) { return t == DR_F32 || t == DR_BF16; }
 template <typename Tin, typename Tout>
 cudaError_t decode_dispatch(int dk, int dv, const void *q, const void *k, const void *v,
                             const float *g, const float *beta, float *state, int B, int Hqk,
-                            int Hv, float scale, void *o, int l2n, cudaStream_t s) {
+                            int Hv, float scale, void *o, int l2n, int cg, cudaStream_t s) {
 #define DR_DEC(DK, DV)                                                                  \
   if (dk == DK && dv == DV)                                                             \
     return dr::launch_decode<DK, DV, Tin, Tout>(q, k, v, g, beta, state, B, Hqk, Hv, scale, o, \
-                                                l2n, s);
+                                                l2n, cg, s);
 #define DR_DEC_ROW(DK) DR_DEC(DK, 16) DR_DEC(DK, 32) DR_DEC(DK, 64) DR_DEC(DK, 128)
   DR_DEC_ROW(16) DR_DEC_ROW(32) DR_DEC_ROW(64) DR_DEC_ROW(128)
 #undef DR_DEC_ROW
@@ -66,7 +66,7 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
                        dr_dtype o_dtype, float *state_out, float *chunk_states,
                        uint32_t flags, dr_stream stream) {
   if (!dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return DR_ERR_DTYPE;
-  if (flags & ~DR_QK_L2NORM) return DR_ERR_UNSUPPORTED;
+  if (flags & ~(DR_QK_L2NORM | DR_GATE_PER_CHANNEL)) return DR_ERR_UNSUPPORTED;
   if (B < 0 || T < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return DR_ERR_SHAPE;
   if (Hv % Hqk != 0) return DR_ERR_SHAPE;
   if (cu_seqlens && (B != 1 || n_seqs < 0)) return DR_ERR_SHAPE;
@@ -74,7 +74,8 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
   if (!std::isfinite(scale)) return DR_ERR_UNSUPPORTED;
   const int64_t N = cu_seqlens ? n_seqs : B;
   const bool tokens = (int64_t)B * T > 0;
-  if (tokens && (!q || !k || !v || !beta || !o)) return DR_ERR_NULL;
+  const bool cg = (flags & DR_GATE_PER_CHANNEL) != 0;
+  if (tokens && (!q || !k || !v || !beta || !o || (cg && !g))) return DR_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(chunk_states, 16) ||
       !aligned(g, 4) ||
@@ -85,9 +86,10 @@ dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float 
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   dr::PrefillArgs a{q, k, v, g, beta, state_in, cu_seqlens, (int)N, B, T, Hqk, Hv,
-                    scale, o, state_out, (flags & DR_QK_L2NORM) ? 1 : 0, chunk_states};
+                    scale, o, state_out, (flags & DR_QK_L2NORM) ? 1 : 0, chunk_states,
+                    cg ? 1 : 0};
   cudaError_t e;
-  if (in_dtype == DR_BF16 && dr::tc_supported(dk, dv)) {
+  if (in_dtype == DR_BF16 && dr::tc_supported(dk, dv) && !cg) {
     e = dr::prefill_tc_dispatch(dk, dv, o_dtype == DR_F32, a, (int)N, s);
   } else if (in_dtype == DR_F32) {
     e = simt_dispatch_out<float>(o_dtype, dk, dv, a, (int)N, s);
@@ -103,13 +105,14 @@ dr_status dr_recurrent_step(const void *q, const void *k, const void *v, const f
                             float scale, void *o, dr_dtype o_dtype, uint32_t flags,
                             dr_stream stream) {
   if (!dtype_ok(in_dtype) || !dtype_ok(o_dtype)) return DR_ERR_DTYPE;
-  if (flags & ~DR_QK_L2NORM) return DR_ERR_UNSUPPORTED;
+  if (flags & ~(DR_QK_L2NORM | DR_GATE_PER_CHANNEL)) return DR_ERR_UNSUPPORTED;
   if (B < 0 || Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return DR_ERR_SHAPE;
   if (Hv % Hqk != 0) return DR_ERR_SHAPE;
   if (!dim_ok(dk) || !dim_ok(dv)) return DR_ERR_UNSUPPORTED;
   if (!std::isfinite(scale)) return DR_ERR_UNSUPPORTED;
   if (B == 0) return DR_OK;
-  if (!q || !k || !v || !beta || !state || !o) return DR_ERR_NULL;
+  const int cg = (flags & DR_GATE_PER_CHANNEL) ? 1 : 0;
+  if (!q || !k || !v || !beta || !state || !o || (cg && !g)) return DR_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(state, 16) || !aligned(g, 4) || !aligned(beta, 4))
     return DR_ERR_ALIGN;
@@ -119,12 +122,12 @@ dr_status dr_recurrent_step(const void *q, const void *k, const void *v, const f
   cudaError_t e;
   if (in_dtype == DR_BF16)
     e = o_dtype == DR_F32
-            ? decode_dispatch<__nv_bfloat16, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, s)
-            : decode_dispatch<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, s);
+            ? decode_dispatch<__nv_bfloat16, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, cg, s)
+            : decode_dispatch<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, cg, s);
   else
     e = o_dtype == DR_F32
-            ? decode_dispatch<float, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, s)
-            : decode_dispatch<float, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, s);
+            ? decode_dispatch<float, float>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, cg, s)
+            : decode_dispatch<float, __nv_bfloat16>(dk, dv, q, k, v, g, beta, state, B, Hqk, Hv, scale, o, l2n, cg, s);
   return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 

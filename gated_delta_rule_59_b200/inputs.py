@@ -20,6 +20,10 @@ heads] float32):
      cached fp32 state ~ N(0, 0.02^2), 64 consecutive steps with fresh inputs
   4  varlen gated prefill: 8 lengths uniform in [512, 16384] + one of 65536,
      packed with cu_seqlens (B=1), H=16 d=128, bf16, g/beta/state as in 2
+
+Per-key-channel gates (``channel_gates=True``, the "linear_attention" page's
+ChannelGates [batch, seq, heads, key_dim]) draw g per channel from the same
+distribution as the scalar gate, in place of it.
 """
 from __future__ import annotations
 
@@ -36,7 +40,7 @@ class Prefill:
     q: torch.Tensor  # [B, T, Hqk, dk]
     k: torch.Tensor  # [B, T, Hqk, dk]
     v: torch.Tensor  # [B, T, Hv, dv]
-    g: Optional[torch.Tensor]  # [B, T, Hv] float32 or None (no decay)
+    g: Optional[torch.Tensor]  # [B, T, Hv] (or [B, T, Hv, dk]: per key channel) float32 or None
     beta: torch.Tensor  # [B, T, Hv] float32
     state_in: Optional[torch.Tensor]  # [N, Hv, dk, dv] float32 or None
     cu_seqlens: Optional[torch.Tensor]  # int32 [N+1] or None
@@ -73,14 +77,14 @@ def _log_sigmoid_gate(gen, shape):
 
 
 def prefill(B, T, Hqk, Hv, dk, dv, dtype=torch.bfloat16, gated=True, beta_max=1.0,
-            state_std=0.0, seed=0, cu_seqlens=None, name="") -> Prefill:
+            state_std=0.0, seed=0, cu_seqlens=None, name="", channel_gates=False) -> Prefill:
     """Generic seeded prefill problem (the shapes and distributions above)."""
     gen = _gen(seed)
     q = _qk(gen, (B, T, Hqk, dk), dtype)
     k = _qk(gen, (B, T, Hqk, dk), dtype)
     v = torch.randn((B, T, Hv, dv), generator=gen).to(dtype)
     beta = (beta_max * torch.sigmoid(torch.randn((B, T, Hv), generator=gen))).float()
-    g = _log_sigmoid_gate(gen, (B, T, Hv)) if gated else None
+    g = _log_sigmoid_gate(gen, (B, T, Hv) + ((dk,) if channel_gates else ())) if gated else None
     N = B if cu_seqlens is None else len(cu_seqlens) - 1
     state = None
     if state_std > 0:
@@ -128,7 +132,7 @@ class DecodeStep:
     q: torch.Tensor  # [B, Hqk, dk]
     k: torch.Tensor  # [B, Hqk, dk]
     v: torch.Tensor  # [B, Hv, dv]
-    g: Optional[torch.Tensor]  # [B, Hv]
+    g: Optional[torch.Tensor]  # [B, Hv] (or [B, Hv, dk]: per key channel)
     beta: torch.Tensor  # [B, Hv]
 
     def to(self, device):
@@ -142,7 +146,7 @@ def decode_state(B, Hv, dk, dv, std=0.02, seed=0) -> torch.Tensor:
 
 
 def decode_steps(B, Hqk, Hv, dk, dv, n_steps, dtype=torch.bfloat16, gated=True,
-                 beta_max=2.0, seed=0):
+                 beta_max=2.0, seed=0, channel_gates=False):
     """``n_steps`` fresh seeded decode inputs (one token per sequence each)."""
     gen = _gen(seed + 1)
     out = []
@@ -151,7 +155,7 @@ def decode_steps(B, Hqk, Hv, dk, dv, n_steps, dtype=torch.bfloat16, gated=True,
         k = _qk(gen, (B, Hqk, dk), dtype)
         v = torch.randn((B, Hv, dv), generator=gen).to(dtype)
         beta = (beta_max * torch.sigmoid(torch.randn((B, Hv), generator=gen))).float()
-        g = _log_sigmoid_gate(gen, (B, Hv)) if gated else None
+        g = _log_sigmoid_gate(gen, (B, Hv) + ((dk,) if channel_gates else ())) if gated else None
         out.append(DecodeStep(q, k, v, g, beta))
     return out
 

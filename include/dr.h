@@ -71,6 +71,11 @@ typedef struct CUstream_st *dr_stream;
                            first (an all-zero row stays zero): the pages' qk_l2norm step
                            ("DeltaNet Attention": queries and keys are L2-normalised before
                            the rule), folded into the kernels as fp32 row and column scalings */
+#define DR_GATE_PER_CHANNEL 2u /* g holds one log decay per key channel, [.., Hv, dk] f32: the
+                                  "linear_attention" page's ChannelGates (its KDA subclass).
+                                  Row i of the stored state decays by exp(g[i]) before the
+                                  write.  g must not be NULL.  dr_chunk_fwd then always runs
+                                  the CUDA-core kernel (fp32 arithmetic) */
 
 /*
  * dr_chunk_fwd -- prompt (prefill) pass: the "chunked rule on a prompt" of the
@@ -81,7 +86,8 @@ typedef struct CUstream_st *dr_stream;
  *   q, k       [B, T, Hqk, dk]   in_dtype (DR_BF16 or DR_F32); L2-normalised by the caller,
  *                                or by the kernel with DR_QK_L2NORM in flags
  *   v          [B, T, Hv, dv]    in_dtype
- *   g          [B, T, Hv] f32    log decay (<= 0 expected); NULL => no decay (plain DeltaNet)
+ *   g          [B, T, Hv] f32    log decay (<= 0 expected); NULL => no decay (plain DeltaNet);
+ *                                [B, T, Hv, dk] with DR_GATE_PER_CHANNEL
  *   beta       [B, T, Hv] f32    write strength
  *   state_in   [N, Hv, dk, dv] f32 or NULL (=> zero state: a fresh prompt).  Read only.
  *   cu_seqlens device int32 [n_seqs + 1] or NULL.  If given, B must be 1, N = n_seqs,
@@ -101,7 +107,7 @@ typedef struct CUstream_st *dr_stream;
  *              min((j + 1) DR_CHUNK, len_n) tokens, and its last row equals its
  *              state_out.  Caller-owned, 16-byte aligned, overlapping no other
  *              argument; rows of a sequence that a bad cu_seqlens skips are not written.
- *   flags      0 or DR_QK_L2NORM
+ *   flags      0 or an OR of DR_QK_L2NORM and DR_GATE_PER_CHANNEL
  *   T = 0 or N = 0 is valid: nothing is read from q/k/v; state_out (if given) receives
  *   state_in (or zeros).
  */
@@ -113,7 +119,8 @@ DR_API dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const
                               float *state_out, float *chunk_states, uint32_t flags,
                               dr_stream stream);
 
-/* Which prefill kernel dr_chunk_fwd launches for these inputs (host only, no device call). */
+/* Which prefill kernel dr_chunk_fwd launches for these inputs without DR_GATE_PER_CHANNEL
+   (host only, no device call); with it the kernel is always DR_KERNEL_SIMT_F32. */
 typedef enum {
   DR_KERNEL_NONE = 0,     /* unsupported dtype / head dimensions                  */
   DR_KERNEL_SIMT_F32 = 1, /* CUDA-core kernel, fp32 arithmetic                    */
@@ -130,7 +137,8 @@ DR_API dr_kernel dr_chunk_fwd_kernel(dr_dtype in_dtype, int32_t dk, int32_t dv);
  * which is the retrieve-and-replace form of the "DeltaNet" page ("The Delta Rule").
  *
  *   q, k   [B, Hqk, dk] in_dtype;   v [B, Hv, dv] in_dtype
- *   g      [B, Hv] f32 or NULL;     beta [B, Hv] f32
+ *   g      [B, Hv] f32 or NULL ([B, Hv, dk] with DR_GATE_PER_CHANNEL: H' = diag(alpha) H);
+ *   beta   [B, Hv] f32
  *   state  [B, Hv, dk, dv] f32, read and overwritten in place
  *   o      [B, Hv, dv] o_dtype
  */
@@ -139,6 +147,7 @@ DR_API dr_status dr_recurrent_step(const void *q, const void *k, const void *v,
                                    int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv,
                                    dr_dtype in_dtype, float scale, void *o, dr_dtype o_dtype,
                                    uint32_t flags, dr_stream stream);
+/* flags of dr_recurrent_step: 0 or an OR of DR_QK_L2NORM and DR_GATE_PER_CHANNEL. */
 
 /* Static English description of a status code (never NULL). */
 DR_API const char *dr_status_string(dr_status status);

@@ -87,8 +87,12 @@ def test_chunk_fwd_argument_errors(L):
     assert chunk(L, cs=ctypes.c_void_p(0x10008)) == 4
     assert chunk(L, cs=P16, B=0) == 0
     # option bits: DR_QK_L2NORM (1) is known, any other bit is unsupported
-    assert chunk(L, flags=2) == 5
+    assert chunk(L, flags=4) == 5
     assert chunk(L, flags=0x80000001) == 5
+    # DR_GATE_PER_CHANNEL (2) needs g
+    assert chunk(L, flags=2) == 1
+    assert chunk(L, flags=3, g=None) == 1
+    assert chunk(L, flags=2, B=0) == 0
     assert chunk(L, B=0, flags=1) == 0
     # nothing to do: no sequences => OK without touching the device
     assert chunk(L, B=0) == 0
@@ -107,13 +111,18 @@ def test_recurrent_step_argument_errors(L):
     assert step(L, o=ctypes.c_void_p(0x10004)) == 4
     assert step(L, g=ctypes.c_void_p(0x10001)) == 4
     assert step(L, flags=4) == 5
+    assert step(L, flags=2) == 1
+    assert step(L, flags=2, B=0) == 0
     assert step(L, B=0, flags=1) == 0
     assert step(L, B=0) == 0
 
 
 def test_chunk_state_rows():
     assert dr.CHUNK == 64
-    assert int(re.search(r"#define DR_CHUNK (\d+)", open(HEADER).read()).group(1)) == dr.CHUNK
+    hdr = open(HEADER).read()
+    assert int(re.search(r"#define DR_CHUNK (\d+)", hdr).group(1)) == dr.CHUNK
+    assert int(re.search(r"#define DR_QK_L2NORM (\d+)u", hdr).group(1)) == dr.QK_L2NORM
+    assert int(re.search(r"#define DR_GATE_PER_CHANNEL (\d+)u", hdr).group(1)) == dr.GATE_PER_CHANNEL
     assert dr.chunk_state_rows(None, 3, 130) == 9
     assert dr.chunk_state_rows(None, 2, 0) == 0
     assert dr.chunk_state_rows([0, 64, 64, 65, 200], 1, 200) == 1 + 0 + 1 + 3
