@@ -6,7 +6,7 @@
 //     H' = alpha H;  v_old = H'^T k;  delta = beta (v - v_old)
 //     H  = H' + k delta^T;            o = H^T q = alpha H^T q + (q.k) delta
 // with H = S^T stored [dk, dv] fp32 (dv contiguous) per (batch, v-head).
-// Per-key-channel gates (cg, g [B, Hv, dk]): H' = diag(alpha) H, so alpha_i folds
+// Per-key-channel gates (CG, g [B, Hv, dk]): H' = diag(alpha) H, so alpha_i folds
 // into k_i and q_i for the two reductions and scales row i of the update.
 //
 // The step is bound by HBM: each (b, h) state is read once and written once
@@ -32,15 +32,17 @@ struct DecodeShape {
   static_assert(DV % 4 == 0 && DK % RP == 0, "unsupported decode shape");
 };
 
-template <int DK, int DV, typename Tin, typename Tout>
+// CG: per-key-channel gates, a compile-time switch so that the scalar-gate kernel carries
+// none of its code.
+template <int DK, int DV, typename Tin, typename Tout, bool CG>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
     decode_step_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k,
                        const Tin *__restrict__ v, const float *__restrict__ g,
                        const float *__restrict__ beta, float *__restrict__ state, int Hqk,
-                       int Hv, float scale, Tout *__restrict__ o, int l2n, int cg) {
+                       int Hv, float scale, Tout *__restrict__ o, int l2n) {
   using S = DecodeShape<DK, DV>;
   constexpr int C4 = S::C4, RP = S::RP, NT = S::NT, RPT = S::RPT;
-  __shared__ float ks[DK], qs[DK], alc[DK];  // alc: per-channel decay (cg)
+  __shared__ float ks[DK], qs[DK], alc[CG ? DK : 1];  // alc: per-channel decay
   __shared__ float4 red_k[RP][C4], red_q[RP][C4];
   __shared__ float qk_shared, nrm[2];
 
@@ -59,7 +61,7 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
   for (int i = t; i < DK; i += NT) {
     ks[i] = io<Tin>::ld(k + qk_off + i);
     qs[i] = scale * io<Tin>::ld(q + qk_off + i);
-    if (cg) alc[i] = expf(g[(size_t)unit * DK + i]);
+    if constexpr (CG) alc[i] = expf(g[(size_t)unit * DK + i]);
   }
   __syncthreads();
   if (l2n) {  // k and q (= scale q) rows divided by their norms; zero rows stay zero
@@ -88,8 +90,11 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
   float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
 #pragma unroll
   for (int i = 0; i < RPT; ++i) {
-    const float ar = cg ? alc[r0 + i * RP] : 1.f;  // exact 1 without channel gates
-    const float kr = ar * ks[r0 + i * RP], qr = ar * qs[r0 + i * RP];
+    float kr = ks[r0 + i * RP], qr = qs[r0 + i * RP];
+    if constexpr (CG) {
+      kr *= alc[r0 + i * RP];
+      qr *= alc[r0 + i * RP];
+    }
     pk.x += kr * hr[i].x; pk.y += kr * hr[i].y; pk.z += kr * hr[i].z; pk.w += kr * hr[i].w;
     pq.x += qr * hr[i].x; pq.y += qr * hr[i].y; pq.z += qr * hr[i].z; pq.w += qr * hr[i].w;
   }
@@ -103,7 +108,7 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
     sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
     sq.x += c.x; sq.y += c.y; sq.z += c.z; sq.w += c.w;
   }
-  const float alpha = (g && !cg) ? expf(g[unit]) : 1.f;
+  const float alpha = (g && !CG) ? expf(g[unit]) : 1.f;
   const float bt = beta[unit];
   const size_t vo = (size_t)unit * DV + 4 * c4;
   float4 d;
@@ -113,7 +118,9 @@ __global__ void __launch_bounds__(DecodeShape<DK, DV>::NT)
   d.w = bt * (io<Tin>::ld(v + vo + 3) - alpha * sk.w);
 #pragma unroll
   for (int i = 0; i < RPT; ++i) {
-    const float kr = ks[r0 + i * RP], ar = cg ? alc[r0 + i * RP] : alpha;
+    const float kr = ks[r0 + i * RP];
+    float ar = alpha;
+    if constexpr (CG) ar = alc[r0 + i * RP];
     float4 nh;
     nh.x = ar * hr[i].x + kr * d.x;
     nh.y = ar * hr[i].y + kr * d.y;
@@ -135,9 +142,11 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
                           const float *beta, float *state, int B, int Hqk, int Hv, float scale,
                           void *o, int l2n, int cg, cudaStream_t stream) {
   const unsigned units = (unsigned)B * (unsigned)Hv;
-  decode_step_kernel<DK, DV, Tin, Tout><<<units, DecodeShape<DK, DV>::NT, 0, stream>>>(
+  auto kern = cg ? decode_step_kernel<DK, DV, Tin, Tout, true>
+                 : decode_step_kernel<DK, DV, Tin, Tout, false>;
+  kern<<<units, DecodeShape<DK, DV>::NT, 0, stream>>>(
       (const Tin *)q, (const Tin *)k, (const Tin *)v, g, beta, state, Hqk, Hv, scale, (Tout *)o,
-      l2n, cg);
+      l2n);
   return cudaGetLastError();
 }
 
