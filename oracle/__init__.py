@@ -11,6 +11,8 @@ Contents
                    q/k L2 normalisation first (``l2_normalize_rows``).
   chunk_ref        numpy fp64 chunk (UT/WY) form, used to pin the chunk algebra.
   brute            exact rational brute force on tiny inputs.
+  layer            prologue and epilogue around the rule: short causal depthwise
+                   convolution + SiLU, RMSNorm / LayerNorm + SiLU output gate.
 
 Parity pins live in ``tests/test_oracle_*.py``.  Every function here is pinned:
 the three forms against one another, against exact rational arithmetic
