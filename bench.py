@@ -359,6 +359,8 @@ def run_ours(args, dist: Dist):
         del cs
         secondary["prefill_channel_gates"] = bench_channel_gates(dev, dist, stream, flush,
                                                                 hbm_peak, peak_kind, args)
+        secondary["prologue_conv_silu"], secondary["epilogue_norm_gate"] = bench_layer_steps(
+            dev, dist, stream, flush, hbm_peak, peak_kind)
         secondary["decode"] = bench_decode(dev, dist, stream, hbm_peak, peak_kind)
         secondary["varlen"] = bench_varlen(dev, dist, stream, flush, hbm_peak, peak_kind)
     clk = clocks.stop()
@@ -416,6 +418,54 @@ def bench_channel_gates(dev, dist, stream, flush, hbm_peak, peak_kind, args):
                      "algorithmic_bytes_per_launch": algo, "peak_kind": peak_kind},
         "gpu_launches": 3,
     }
+
+
+def bench_layer_steps(dev, dist, stream, flush, hbm_peak, peak_kind):
+    """The steps either side of the rule on the headline shapes (bf16 activations):
+    conv + SiLU of q, k, v (K = 4, conv state out), and RMSNorm + SiLU gate of o (fp32) with
+    z (bf16) into bf16.  Both are HBM bound: bytes = every element read and written once."""
+    import gated_delta_rule_59_b200 as dr
+
+    B, T, Hqk, Hv, d, K = 2, 8192, 16, 32, 128, 4
+    gen = torch.Generator().manual_seed(77)
+    xs = [torch.randn((B, T, H, d), generator=gen).to(torch.bfloat16).to(dev)
+          for H in (Hqk, Hqk, Hv)]
+    ws = [(0.5 * torch.randn((H, d, K), generator=gen)).to(dev) for H in (Hqk, Hqk, Hv)]
+    o = torch.randn((B, T, Hv, d), generator=gen).to(dev)
+    z = torch.randn((B, T, Hv, d), generator=gen).to(torch.bfloat16).to(dev)
+    wt = torch.ones(d, device=dev)
+    y = torch.empty((B, T, Hv, d), dtype=torch.bfloat16, device=dev)
+
+    def conv_step(_):
+        for x, w in zip(xs, ws):
+            dr.short_conv_silu(x, w)
+
+    def norm_step(_):
+        dr.norm_gate(o, wt, z=z, y=y)
+
+    out = []
+    for fn, nbytes, launches, metric in (
+            (conv_step, sum(4 * x.numel() + B * x[0, 0].numel() * (K - 1) * 4 for x in xs), 6,
+             "conv + SiLU of q, k, v (K=4) on the headline shape, bf16 in and out"),
+            (norm_step, o.numel() * 4 + z.numel() * 2 + y.numel() * 2, 1,
+             "RMSNorm + SiLU gate of o (fp32) with z (bf16) into bf16, headline shape")):
+        for i in range(3):
+            flush.zero_()
+            fn(i)
+        torch.cuda.synchronize()
+        assert dr.device_status(dev) == 0
+        dist.barrier()
+        durs = time_steps(fn, 10, stream, flush)
+        dist.barrier()
+        ms = dist.max(sum(durs) / len(durs), dev)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out.append({"metric": metric, "value": round(gbs, 1), "unit": "GB/s",
+                    "ms_per_step": round(ms, 4), "gpu_launches": 10 * launches,
+                    "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak,
+                                 "frac": round(gbs / hbm_peak, 4), "unit": "GB/s",
+                                 "algorithmic_bytes_per_step": nbytes,
+                                 "peak_kind": peak_kind}})
+    return out[0], out[1]
 
 
 def bench_decode(dev, dist, stream, hbm_peak, peak_kind):

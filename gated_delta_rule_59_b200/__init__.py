@@ -3,23 +3,26 @@
 This module only marshals arguments: it checks tensor placement, dtype and
 contiguity, allocates outputs with PyTorch (device memory and streams are the
 only things PyTorch does here) and passes raw device pointers plus the current
-CUDA stream to ``dr_chunk_fwd`` / ``dr_recurrent_step`` (``include/dr.h``).
-Every step of the recurrence runs in the library's CUDA kernels; there is no
-CPU or PyTorch fallback, and a missing or unloadable ``libdr.so`` raises.
+CUDA stream to the library's calls (``include/dr.h``).  Every step runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and a missing or
+unloadable ``libdr.so`` raises.
 
     o, state_out = chunk_fwd(q, k, v, g, beta, state_in=None, cu_seqlens=None)
     o = recurrent_step(q, k, v, g, beta, state)      # state updated in place
+    y, conv_state = short_conv_silu(x, w)            # the step before the rule
+    out = norm_gate(o, weight, z=z)                  # the step after it
 """
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Optional
 
 import torch
 
-__all__ = ["chunk_fwd", "recurrent_step", "device_status", "prefill_kernel", "chunk_state_rows",
-           "lib", "DrError", "LIB_PATH", "CHUNK"]
+__all__ = ["chunk_fwd", "recurrent_step", "short_conv_silu", "norm_gate", "device_status",
+           "prefill_kernel", "chunk_state_rows", "lib", "DrError", "LIB_PATH", "CHUNK"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdr.so")
 
@@ -51,6 +54,12 @@ def lib() -> ctypes.CDLL:
                                    ctypes.c_int, ctypes.c_float, vp, ctypes.c_int, fp, fp,
                                    ctypes.c_uint32, vp]
         L.dr_chunk_fwd.restype = ctypes.c_int
+        L.dr_short_conv_silu.argtypes = [vp, ctypes.c_int, fp, i32, fp, fp, ip, i32, i32, i32,
+                                         i32, vp, ctypes.c_int, vp]
+        L.dr_short_conv_silu.restype = ctypes.c_int
+        L.dr_norm_gate.argtypes = [vp, ctypes.c_int, fp, fp, vp, ctypes.c_int, ctypes.c_int64,
+                                   i32, i32, ctypes.c_float, vp, ctypes.c_int, vp]
+        L.dr_norm_gate.restype = ctypes.c_int
         L.dr_recurrent_step.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, i32,
                                         ctypes.c_int, ctypes.c_float, vp, ctypes.c_int,
                                         ctypes.c_uint32, vp]
@@ -204,6 +213,84 @@ def recurrent_step(q, k, v, g, beta, state, scale: float = 1.0, out_dtype=torch.
     if rc != 0:
         raise DrError(rc, "dr_recurrent_step")
     return o
+
+
+def short_conv_silu(x, w, conv_state=None, cu_seqlens=None, out_dtype=None,
+                    output_conv_state: bool = True):
+    """Causal depthwise convolution + SiLU through ``dr_short_conv_silu``.
+
+    x [B, T, H, d] (or [B, T, C]) bf16 or fp32; w [H, d, K] (or [C, K]) fp32, K <= 8;
+    conv_state [N, H, d, K-1] fp32 or None (zero history); cu_seqlens int32 [N+1] or None.
+    Returns (y like x in ``out_dtype`` (default x's dtype), conv_state_out or None).
+    """
+    if x.dtype not in _DTYPES:
+        raise ValueError("x must be bf16 or fp32")
+    out_dtype = x.dtype if out_dtype is None else out_dtype
+    if out_dtype not in _DTYPES:
+        raise ValueError("out_dtype must be bf16 or fp32")
+    dev = x.device
+    _check(x, "x", x.dtype, dev)
+    _check(w, "w", torch.float32, dev)
+    _check(conv_state, "conv_state", torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    B, T = x.shape[:2]
+    C = math.prod(x.shape[2:])
+    K = w.shape[-1]
+    if w.numel() != C * K:
+        raise ValueError("w must hold K taps per channel of x")
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if conv_state is not None and conv_state.numel() != N * C * (K - 1):
+        raise ValueError("conv_state must be [N, channels, K-1]")
+    y = torch.empty(x.shape, dtype=out_dtype, device=dev)
+    st = (torch.empty((N,) + tuple(x.shape[2:]) + (K - 1,), dtype=torch.float32, device=dev)
+          if output_conv_state else None)
+    rc = lib().dr_short_conv_silu(
+        _ptr(x), _DTYPES[x.dtype], _ptr(w), K, _ptr(conv_state), _ptr(st), _ptr(cu_seqlens),
+        N, B, T, C, _ptr(y), _DTYPES[out_dtype], _stream(dev))
+    if rc != 0:
+        raise DrError(rc, "dr_short_conv_silu")
+    return y, st
+
+
+NORM_KINDS = {"rms": 0, "layer": 1}  # DR_NORM_RMS, DR_NORM_LAYER of include/dr.h
+
+
+def norm_gate(o, weight, bias=None, z=None, kind: str = "rms", eps=None, out_dtype=None, y=None):
+    """Per-(token, head) RMSNorm / LayerNorm over the last axis, then y * silu(z)
+    through ``dr_norm_gate``.
+
+    o [..., dv] bf16 or fp32 (dv <= 128); weight, bias [dv] fp32 (bias: LayerNorm only, or
+    None); z like o (any of the two dtypes) or None.  eps defaults to 1e-6 (RMSNorm) or 1e-5
+    (LayerNorm).  ``y`` may be ``o`` itself (in place) when the dtypes match; the output
+    dtype is ``out_dtype``, else y's, else o's.
+    """
+    if o.dtype not in _DTYPES:
+        raise ValueError("o must be bf16 or fp32")
+    if out_dtype is None:
+        out_dtype = o.dtype if y is None else y.dtype
+    dev = o.device
+    _check(o, "o", o.dtype, dev)
+    _check(weight, "weight", torch.float32, dev)
+    _check(bias, "bias", torch.float32, dev)
+    if z is not None:
+        _check(z, "z", z.dtype, dev)
+        if z.dtype not in _DTYPES or z.shape != o.shape:
+            raise ValueError("z must be bf16 or fp32 and shaped like o")
+    dv = o.shape[-1]
+    if weight.numel() != dv or (bias is not None and bias.numel() != dv):
+        raise ValueError("weight / bias must have dv entries")
+    if y is None:
+        y = torch.empty(o.shape, dtype=out_dtype, device=dev)
+    _check(y, "y", out_dtype, dev)
+    if eps is None:
+        eps = 1e-6 if kind == "rms" else 1e-5
+    rc = lib().dr_norm_gate(
+        _ptr(o), _DTYPES[o.dtype], _ptr(weight), _ptr(bias), _ptr(z),
+        _DTYPES[z.dtype] if z is not None else 0, o.numel() // dv, dv, NORM_KINDS[kind],
+        float(eps), _ptr(y), _DTYPES[out_dtype], _stream(dev))
+    if rc != 0:
+        raise DrError(rc, "dr_norm_gate")
+    return y
 
 
 KERNELS = {0: None, 1: "simt_f32", 2: "tc_bf16"}

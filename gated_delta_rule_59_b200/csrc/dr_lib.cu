@@ -13,6 +13,7 @@
 #include "chunk_simt.cuh"
 #include "chunk_tc.cuh"
 #include "chunk_pair.cuh"
+#include "layer.cuh"
 
 #define DR_VERSION_NUMBER 100  // 0.1.0
 
@@ -55,9 +56,119 @@ cudaError_t simt_dispatch_out(dr_dtype od, int dk, int dv, const dr::PrefillArgs
                       : simt_dispatch<Tin, __nv_bfloat16>(dk, dv, a, N, s);
 }
 
+template <typename Tin, typename Tout>
+cudaError_t launch_conv(const void *x, const float *w, int K, const float *state_in,
+                        const int32_t *cu, int n_seqs, int T, long long P, int C, void *y,
+                        cudaStream_t s) {
+  if (P == 0) return cudaSuccess;
+  const dim3 grid((unsigned)((P + dr::CONV_TOK - 1) / dr::CONV_TOK), (unsigned)((C + 127) / 128));
+  dr::conv_silu_kernel<Tin, Tout><<<grid, 128, 0, s>>>((const Tin *)x, w, K, state_in, cu,
+                                                       cu ? n_seqs : 1, T, P, C, (Tout *)y);
+  return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t conv_dispatch_out(dr_dtype yd, const void *x, const float *w, int K,
+                              const float *state_in, const int32_t *cu, int n_seqs, int T,
+                              long long P, int C, void *y, cudaStream_t s) {
+  return yd == DR_F32 ? launch_conv<Tin, float>(x, w, K, state_in, cu, n_seqs, T, P, C, y, s)
+                      : launch_conv<Tin, __nv_bfloat16>(x, w, K, state_in, cu, n_seqs, T, P, C, y, s);
+}
+
+template <typename Tin>
+cudaError_t launch_conv_state(const void *x, int K, const float *state_in, const int32_t *cu,
+                              int n_seqs, int N, int T, int C, float *state_out, cudaStream_t s) {
+  const long long threads = (long long)N * C;
+  if (threads == 0 || K == 1) return cudaSuccess;
+  dr::conv_state_kernel<Tin><<<(unsigned)((threads + 127) / 128), 128, 0, s>>>(
+      (const Tin *)x, K, state_in, cu, n_seqs, N, T, C, state_out);
+  return cudaGetLastError();
+}
+
+template <typename Tin, typename Tz>
+cudaError_t norm_dispatch_out(dr_dtype yd, const void *o, const float *wt, const float *bias,
+                              const void *z, long long rows, int dv, int layer, float eps, void *y,
+                              cudaStream_t s) {
+  const unsigned blocks = (unsigned)((rows + 7) / 8);
+  if (yd == DR_F32)
+    dr::norm_gate_kernel<Tin, Tz, float><<<blocks, 256, 0, s>>>(
+        (const Tin *)o, wt, bias, (const Tz *)z, rows, dv, layer, eps, (float *)y);
+  else
+    dr::norm_gate_kernel<Tin, Tz, __nv_bfloat16><<<blocks, 256, 0, s>>>(
+        (const Tin *)o, wt, bias, (const Tz *)z, rows, dv, layer, eps, (__nv_bfloat16 *)y);
+  return cudaGetLastError();
+}
+
+size_t dsize(dr_dtype t) { return t == DR_F32 ? 4 : 2; }
+
 }  // namespace
 
 extern "C" {
+
+dr_status dr_short_conv_silu(const void *x, dr_dtype x_dtype, const float *w, int32_t K,
+                             const float *conv_state_in, float *conv_state_out,
+                             const int32_t *cu_seqlens, int32_t n_seqs, int32_t B, int32_t T,
+                             int32_t C, void *y, dr_dtype y_dtype, dr_stream stream) {
+  if (!dtype_ok(x_dtype) || !dtype_ok(y_dtype)) return DR_ERR_DTYPE;
+  if (B < 0 || T < 0 || C <= 0 || K < 1) return DR_ERR_SHAPE;
+  if (K > dr::CONV_MAX_K) return DR_ERR_UNSUPPORTED;
+  if (cu_seqlens && (B != 1 || n_seqs < 0)) return DR_ERR_SHAPE;
+  const long long P = (long long)B * T;
+  if (cu_seqlens && n_seqs == 0 && P > 0) return DR_ERR_SHAPE;
+  const int64_t N = cu_seqlens ? n_seqs : B;
+  if (P > 0 && (!x || !w || !y)) return DR_ERR_NULL;
+  if (!aligned(x, dsize(x_dtype)) || !aligned(y, dsize(y_dtype)) || !aligned(w, 4) ||
+      !aligned(conv_state_in, 4) || !aligned(conv_state_out, 4) || !aligned(cu_seqlens, 4))
+    return DR_ERR_ALIGN;
+  if ((P + dr::CONV_TOK - 1) / dr::CONV_TOK > 0x7fffffffLL || (C + 127) / 128 > 65535 ||
+      N * (int64_t)C > 0x3fffffffffLL)
+    return DR_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (x_dtype == DR_F32)
+    e = conv_dispatch_out<float>(y_dtype, x, w, K, conv_state_in, cu_seqlens, n_seqs, T, P, C, y, s);
+  else
+    e = conv_dispatch_out<__nv_bfloat16>(y_dtype, x, w, K, conv_state_in, cu_seqlens, n_seqs, T, P,
+                                         C, y, s);
+  if (e == cudaSuccess && conv_state_out)
+    e = x_dtype == DR_F32
+            ? launch_conv_state<float>(x, K, conv_state_in, cu_seqlens, n_seqs, (int)N, T, C,
+                                       conv_state_out, s)
+            : launch_conv_state<__nv_bfloat16>(x, K, conv_state_in, cu_seqlens, n_seqs, (int)N, T,
+                                               C, conv_state_out, s);
+  return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
+dr_status dr_norm_gate(const void *o, dr_dtype o_dtype, const float *weight, const float *bias,
+                       const void *z, dr_dtype z_dtype, int64_t rows, int32_t dv, int32_t kind,
+                       float eps, void *y, dr_dtype y_dtype, dr_stream stream) {
+  if (!dtype_ok(o_dtype) || !dtype_ok(y_dtype) || (z && !dtype_ok(z_dtype))) return DR_ERR_DTYPE;
+  if (rows < 0 || dv <= 0) return DR_ERR_SHAPE;
+  if (dv > 128 || (kind != DR_NORM_RMS && kind != DR_NORM_LAYER) || !(eps >= 0.f) ||
+      !std::isfinite(eps))
+    return DR_ERR_UNSUPPORTED;
+  if (rows == 0) return DR_OK;
+  if (!o || !weight || !y) return DR_ERR_NULL;
+  if (!aligned(o, dsize(o_dtype)) || !aligned(y, dsize(y_dtype)) || !aligned(weight, 4) ||
+      !aligned(bias, 4) || (z && !aligned(z, dsize(z_dtype))))
+    return DR_ERR_ALIGN;
+  if ((rows + 7) / 8 > 0x7fffffffLL) return DR_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int layer = kind == DR_NORM_LAYER ? 1 : 0;
+  const bool zf = z == nullptr || z_dtype == DR_F32;
+  cudaError_t e;
+  if (o_dtype == DR_F32)
+    e = zf ? norm_dispatch_out<float, float>(y_dtype, o, weight, bias, z, rows, dv, layer, eps, y, s)
+           : norm_dispatch_out<float, __nv_bfloat16>(y_dtype, o, weight, bias, z, rows, dv, layer,
+                                                     eps, y, s);
+  else
+    e = zf ? norm_dispatch_out<__nv_bfloat16, float>(y_dtype, o, weight, bias, z, rows, dv, layer,
+                                                     eps, y, s)
+           : norm_dispatch_out<__nv_bfloat16, __nv_bfloat16>(y_dtype, o, weight, bias, z, rows, dv,
+                                                             layer, eps, y, s);
+  return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
 
 dr_status dr_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                        const float *beta, const float *state_in, const int32_t *cu_seqlens,

@@ -149,6 +149,49 @@ DR_API dr_status dr_recurrent_step(const void *q, const void *k, const void *v,
                                    uint32_t flags, dr_stream stream);
 /* flags of dr_recurrent_step: 0 or an OR of DR_QK_L2NORM and DR_GATE_PER_CHANNEL. */
 
+/*
+ * dr_short_conv_silu -- the step before the rule in the "DeltaNet" layer diagram: a
+ * causal depthwise convolution ("Conv*") of the projected q, k or v, then SiLU:
+ *     y_t[c] = silu(sum_{j<K} w[c][j] x_{t-K+1+j}[c]),   silu(u) = u / (1 + e^-u)
+ * Tap K-1 weighs the current token.  Before a sequence's first token the inputs are the
+ * sequence's conv_state_in (its last K-1 inputs of a previous call, oldest first) or zero;
+ * sequences never see one another.
+ *
+ *   x          [B, T, C] x_dtype (C channels, e.g. heads * head_dim, contiguous)
+ *   w          [C, K] f32, 1 <= K <= 8
+ *   conv_state_in  [N, C, K-1] f32 or NULL (zero history)
+ *   conv_state_out [N, C, K-1] f32 or NULL: the last K-1 inputs of every sequence (history
+ *              included when a sequence is shorter); may be conv_state_in itself
+ *   cu_seqlens as for dr_chunk_fwd (B = 1, N = n_seqs); else N = B sequences of T tokens
+ *   y          [B, T, C] y_dtype; must not overlap x
+ */
+DR_API dr_status dr_short_conv_silu(const void *x, dr_dtype x_dtype, const float *w, int32_t K,
+                                    const float *conv_state_in, float *conv_state_out,
+                                    const int32_t *cu_seqlens, int32_t n_seqs, int32_t B,
+                                    int32_t T, int32_t C, void *y, dr_dtype y_dtype,
+                                    dr_stream stream);
+
+typedef enum { DR_NORM_RMS = 0, DR_NORM_LAYER = 1 } dr_norm_kind;
+
+/*
+ * dr_norm_gate -- the step after the rule: per-(token, head) normalisation of the
+ * readout over its dv values ("DeltaNet": RMSNorm; "DeltaNet Attention": LayerNorm
+ * `norm`), then the SiLU output gate of "DeltaNet Attention" (`g_proj`):
+ *     RMS:    u = o / sqrt(mean(o^2) + eps) * weight
+ *     LAYER:  u = (o - mean(o)) / sqrt(var(o) + eps) * weight + bias   (biased variance)
+ *     y = z ? u * silu(z) : u
+ *
+ *   o       [rows, dv] o_dtype (rows = B * T * Hv), dv <= 128
+ *   weight  [dv] f32;  bias [dv] f32 or NULL (LayerNorm only)
+ *   z       [rows, dv] z_dtype or NULL (no gate)
+ *   y       [rows, dv] y_dtype; may be o itself when the dtypes match
+ *   eps     >= 0 (1e-6 for RMSNorm and 1e-5 for LayerNorm are the usual values)
+ */
+DR_API dr_status dr_norm_gate(const void *o, dr_dtype o_dtype, const float *weight,
+                              const float *bias, const void *z, dr_dtype z_dtype, int64_t rows,
+                              int32_t dv, int32_t kind, float eps, void *y, dr_dtype y_dtype,
+                              dr_stream stream);
+
 /* Static English description of a status code (never NULL). */
 DR_API const char *dr_status_string(dr_status status);
 

@@ -29,10 +29,12 @@ from __future__ import annotations
 
 import numpy as np
 
+from . import _f64  # float64 numpy view of a numpy array or a torch tensor of any dtype
+
 
 def silu(x):
     """x sigmoid(x), evaluated without overflow for large negative x."""
-    x = np.asarray(x, dtype=np.float64)
+    x = _f64(x)
     return np.where(x >= 0, x / (1.0 + np.exp(-np.abs(x))),
                     x * np.exp(-np.abs(x)) / (1.0 + np.exp(-np.abs(x))))
 
@@ -52,8 +54,7 @@ def short_conv_silu(x, w, conv_state=None, cu_seqlens=None):
     silu(sum_j w[c, j] x_{t-K+1+j}[c]), and conv_state_out holds the last K-1 inputs of
     each sequence (history included when the sequence is shorter than K-1).
     """
-    x = np.asarray(x, dtype=np.float64)
-    w = np.asarray(w, dtype=np.float64)
+    x, w = _f64(x), _f64(w)
     B, T, H, d = x.shape
     K = w.shape[-1]
     assert w.shape == (H, d, K)
@@ -62,7 +63,7 @@ def short_conv_silu(x, w, conv_state=None, cu_seqlens=None):
     st_out = np.zeros((len(seqs), H, d, K - 1))
     for n, (b, t0, t1) in enumerate(seqs):
         hist = (np.zeros((K - 1, H, d)) if conv_state is None
-                else np.moveaxis(np.asarray(conv_state[n], dtype=np.float64), -1, 0))
+                else np.moveaxis(_f64(conv_state[n]), -1, 0))
         xp = np.concatenate([hist, x[b, t0:t1]], axis=0)  # [K-1 + L, H, d]
         for t in range(t1 - t0):
             acc = np.zeros((H, d))
@@ -82,8 +83,7 @@ def norm_gate(o, weight, bias=None, z=None, kind="rms", eps=None):
     kind "layer": y = (o - mean(o)) / sqrt(var(o) + eps) * weight + bias  (eps 1e-5)
     then y * silu(z) when z is given.
     """
-    o = np.asarray(o, dtype=np.float64)
-    weight = np.asarray(weight, dtype=np.float64)
+    o, weight = _f64(o), _f64(weight)
     if kind == "rms":
         e = 1e-6 if eps is None else eps
         y = o / np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + e) * weight
@@ -93,7 +93,7 @@ def norm_gate(o, weight, bias=None, z=None, kind="rms", eps=None):
         var = np.mean((o - mu) ** 2, axis=-1, keepdims=True)
         y = (o - mu) / np.sqrt(var + e) * weight
         if bias is not None:
-            y = y + np.asarray(bias, dtype=np.float64)
+            y = y + _f64(bias)
     else:
         raise ValueError(kind)
     if z is not None:

@@ -117,12 +117,37 @@ def test_recurrent_step_argument_errors(L):
     assert step(L, B=0) == 0
 
 
+def test_conv_and_norm_argument_errors(L):
+    conv = lambda x=P16, xd=1, w=P16, K=4, si=None, so=None, cu=None, n=0, B=1, T=8, C=16, \
+        y=P16, yd=1: L.dr_short_conv_silu(x, xd, w, K, si, so, cu, n, B, T, C, y, yd, None)
+    assert conv(xd=5) == 3
+    assert conv(K=0) == 2 and conv(C=0) == 2 and conv(T=-1) == 2
+    assert conv(K=9) == 5
+    assert conv(cu=P16, B=2, n=1) == 2
+    assert conv(cu=P16, n=0) == 2  # tokens but no sequence
+    assert conv(x=None) == 1 and conv(w=None) == 1 and conv(y=None) == 1
+    assert conv(x=ctypes.c_void_p(0x10001)) == 4
+    assert conv(w=ctypes.c_void_p(0x10002)) == 4
+    assert conv(B=0) == 0 and conv(B=0, x=None, y=None) == 0
+    norm = lambda o=P16, od=0, w=P16, b=None, z=None, zd=0, rows=4, dv=64, kind=0, eps=1e-6, \
+        y=P16, yd=0: L.dr_norm_gate(o, od, w, b, z, zd, rows, dv, kind, eps, y, yd, None)
+    assert norm(od=4) == 3 and norm(z=P16, zd=9) == 3
+    assert norm(rows=-1) == 2 and norm(dv=0) == 2
+    assert norm(dv=129) == 5 and norm(kind=2) == 5 and norm(eps=-1.0) == 5
+    assert norm(eps=float("nan")) == 5
+    assert norm(o=None) == 1 and norm(w=None) == 1 and norm(y=None) == 1
+    assert norm(o=ctypes.c_void_p(0x10002)) == 4
+    assert norm(rows=0, o=None) == 0
+
+
 def test_chunk_state_rows():
     assert dr.CHUNK == 64
     hdr = open(HEADER).read()
     assert int(re.search(r"#define DR_CHUNK (\d+)", hdr).group(1)) == dr.CHUNK
     assert int(re.search(r"#define DR_QK_L2NORM (\d+)u", hdr).group(1)) == dr.QK_L2NORM
     assert int(re.search(r"#define DR_GATE_PER_CHANNEL (\d+)u", hdr).group(1)) == dr.GATE_PER_CHANNEL
+    assert re.search(r"DR_NORM_RMS = (\d+), DR_NORM_LAYER = (\d+)", hdr).groups() == (
+        str(dr.NORM_KINDS["rms"]), str(dr.NORM_KINDS["layer"]))
     assert dr.chunk_state_rows(None, 3, 130) == 9
     assert dr.chunk_state_rows(None, 2, 0) == 0
     assert dr.chunk_state_rows([0, 64, 64, 65, 200], 1, 200) == 1 + 0 + 1 + 3
