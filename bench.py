@@ -357,12 +357,15 @@ def run_ours(args, dist: Dist):
                              kfile, "gated_prefill_chunk_states_B2_T8192_Hqk16_Hv32_d128")},
         }
         del cs
-        secondary["prefill_channel_gates"] = bench_channel_gates(dev, dist, stream, flush,
-                                                                hbm_peak, peak_kind, args)
-        secondary["prologue_conv_silu"], secondary["epilogue_norm_gate"] = bench_layer_steps(
-            dev, dist, stream, flush, hbm_peak, peak_kind)
-        secondary["decode"] = bench_decode(dev, dist, stream, hbm_peak, peak_kind)
-        secondary["varlen"] = bench_varlen(dev, dist, stream, flush, hbm_peak, peak_kind)
+        secondary["prefill_channel_gates"] = guarded(bench_channel_gates, dev, dist, stream,
+                                                     flush, hbm_peak, peak_kind, args)
+        layer_lines = guarded(bench_layer_steps, dev, dist, stream, flush, hbm_peak, peak_kind)
+        if isinstance(layer_lines, dict):  # the error record
+            layer_lines = (layer_lines, layer_lines)
+        secondary["prologue_conv_silu"], secondary["epilogue_norm_gate"] = layer_lines
+        secondary["decode"] = guarded(bench_decode, dev, dist, stream, hbm_peak, peak_kind)
+        secondary["varlen"] = guarded(bench_varlen, dev, dist, stream, flush, hbm_peak,
+                                      peak_kind)
     clk = clocks.stop()
 
     line = {
@@ -384,6 +387,15 @@ def run_ours(args, dist: Dist):
     dist.close()
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def guarded(fn, *args):
+    """A secondary line that raises on the host is reported as an error record instead of
+    costing the headline line.  Every rank runs the same code, so all raise at the same point."""
+    try:
+        return fn(*args)
+    except (ValueError, RuntimeError, AssertionError) as e:
+        return {"error": f"{type(e).__name__}: {e}"}
 
 
 def bench_channel_gates(dev, dist, stream, flush, hbm_peak, peak_kind, args):
