@@ -108,3 +108,26 @@ def test_cg5_rows_outside_the_key_support_only_decay():
     # and the channels with keys did take writes
     assert np.max(np.abs(s[0, 0, :3] - np.exp(np.sum(g[0, :, 0, :3], axis=0))[:, None]
                          * s0[0, 0, :3])) > 1e-3
+
+
+def test_golden_exact_fixture_with_chunk_states():
+    """Exact rational values written by tests/golden/make_golden.py (brute force only)."""
+    import json
+    import os
+
+    path = os.path.join(os.path.dirname(__file__), "golden", "brute_channel_gates.json")
+    with open(path) as fh:
+        fx = json.load(fh)
+    F = lambda x: float(Fraction(x))
+    arr = lambda m: np.array([[F(x) for x in row] for row in m])
+    q, k, v, S0 = arr(fx["q"]), arr(fx["k"]), arr(fx["v"]), arr(fx["S0"])
+    g = np.log(arr(fx["alpha"]))
+    beta = np.array([F(b) for b in fx["beta"]])
+    o, st, cs = oracle.run(q[None, :, None], k[None, :, None], v[None, :, None],
+                           g[None, :, None, :], beta[None, :, None], S0.T[None, None],
+                           chunk_len=2)
+    assert rel(o[0, :, 0], arr(fx["o"])) < 1e-13
+    assert rel(st[0, 0], arr(fx["S_T"]).T) < 1e-13
+    for j, S in enumerate(fx["S_after"]):
+        assert rel(cs[j, 0], arr(S).T) < 1e-13
+
